@@ -1,0 +1,428 @@
+"""Pins of the CPU oracle against what the pages and the mathematics fix.
+
+Each test checks the oracle against something other than itself: a closed
+form, a textbook special case of the delta rule, an invariant of the method,
+a hand-derived fixture under tests/golden/, a library routine, or a
+brute-force enumeration on tiny heads.  Together they are meant to fail on a
+dropped term, a wrong sign or index, or a transposed operand anywhere in the
+oracle.  Sources: news post "Linear attention has to move state every token it
+generates; LeapQuant compresses it to 8-bit without losing accuracy" (the
+per-window, Compensator Tokens and residual smoothing paragraphs) and
+"LeapQuant: Efficient Linear Attention with Accurate Recurrent State
+Quantization" (original abstract).
+"""
+import json
+import os
+
+import numpy as np
+import pytest
+
+import oracle
+from tests import brute
+
+GOLDEN = os.path.join(os.path.dirname(__file__), "golden")
+
+
+def _rand_state(rng, dk, dv, rows=(), cols=(), gain=50.0):
+    S = rng.normal(0, 0.1, (dk, dv))
+    for i in rows:
+        S[i] *= gain
+    for j in cols:
+        S[:, j] *= gain
+    return S
+
+
+def _unit(rng, n):
+    x = rng.normal(size=n)
+    return x / np.linalg.norm(x)
+
+
+# --------------------------------------------------------------------------
+# the delta-rule step (GDN / KDA)
+
+def test_step_delta_rule_overwrites_key_row(oracle_lib):
+    """k = e_i, beta = 1: the step writes v into key row i after the decay,
+    every other row is only decayed, and o = S_t^T q with q = e_i returns v."""
+    rng = np.random.default_rng(1)
+    dk, dv = 8, 6
+    S = rng.normal(size=(dk, dv))          # not symmetric, not square
+    a = rng.uniform(0.5, 1.0, dk)
+    i = 3
+    e = np.zeros(dk)
+    e[i] = 1.0
+    v = rng.normal(size=dv)
+    S1, o, u = oracle.step(S, e, e, v, 1.0, a)
+    expect = a[:, None] * S
+    expect[i] = v
+    np.testing.assert_allclose(S1, expect, rtol=0, atol=1e-14)
+    np.testing.assert_allclose(o, v, rtol=0, atol=1e-14)
+    np.testing.assert_allclose(u, v - a[i] * S[i], rtol=0, atol=1e-14)
+
+
+def test_step_beta_zero_is_pure_decay(oracle_lib):
+    rng = np.random.default_rng(2)
+    dk, dv = 8, 8
+    S = rng.normal(size=(dk, dv))
+    a = rng.uniform(0.3, 1.0, dk)
+    q, k, v = _unit(rng, dk), _unit(rng, dk), rng.normal(size=dv)
+    S1, o, u = oracle.step(S, q, k, v, 0.0, a)
+    np.testing.assert_array_equal(S1, a[:, None] * S)
+    np.testing.assert_allclose(o, (a[:, None] * S).T @ q, rtol=1e-13, atol=1e-15)
+    np.testing.assert_array_equal(u, np.zeros(dv))
+
+
+@pytest.mark.parametrize("alpha", [1.0, 0.93])
+def test_step_matches_textbook_gated_delta_rule(oracle_lib, alpha):
+    """Textbook form S_t = alpha (I - beta k k^T) S_{t-1} + beta k v^T
+    (alpha = 1: plain DeltaNet), o_t = S_t^T q_t."""
+    rng = np.random.default_rng(3)
+    dk, dv = 16, 12
+    S = rng.normal(size=(dk, dv))
+    for _ in range(5):
+        q, k, v = _unit(rng, dk), _unit(rng, dk), rng.normal(size=dv)
+        beta = rng.uniform(0.1, 0.9)
+        ref = alpha * (np.eye(dk) - beta * np.outer(k, k)) @ S + beta * np.outer(k, v)
+        S, o, _ = oracle.step(S, q, k, v, beta, np.full(dk, alpha))
+        np.testing.assert_allclose(S, ref, rtol=1e-12, atol=1e-13)
+        np.testing.assert_allclose(o, ref.T @ q, rtol=1e-12, atol=1e-13)
+
+
+def test_step_matches_textbook_kda(oracle_lib):
+    """KDA: S_t = (I - beta k k^T) diag(a) S_{t-1} + beta k v^T."""
+    rng = np.random.default_rng(4)
+    dk, dv = 16, 8
+    S = rng.normal(size=(dk, dv))
+    for _ in range(5):
+        q, k, v = _unit(rng, dk), _unit(rng, dk), rng.normal(size=dv)
+        a = rng.uniform(0.4, 1.0, dk)
+        beta = rng.uniform(0.1, 0.9)
+        ref = (np.eye(dk) - beta * np.outer(k, k)) @ np.diag(a) @ S + beta * np.outer(k, v)
+        S, o, _ = oracle.step(S, q, k, v, beta, a)
+        np.testing.assert_allclose(S, ref, rtol=1e-12, atol=1e-13)
+        np.testing.assert_allclose(o, ref.T @ q, rtol=1e-12, atol=1e-13)
+
+
+def test_kda_with_uniform_decay_is_gdn(oracle_lib):
+    from linear_attention_recurrent_lq_b200 import inputs
+    wl = inputs.WORKLOADS["gdn_int8_b1h1"].replace(tokens=40)
+    d = inputs.draw(wl)
+    nh = 1
+    S0 = d["S0"].reshape(nh, 128, 128)
+    q, k, v = (d[x].reshape(40, nh, 128) for x in "qkv")
+    beta = d["beta"].reshape(40, nh)
+    alpha = d["decay"].reshape(40, nh)
+    pg = oracle.Params.of(wl)
+    pk = oracle.Params(**{**pg.__dict__, "kda": True})
+    og, Sg, _ = oracle.run(pg, S0, q, k, v, beta, alpha)
+    ok, Sk, _ = oracle.run(pk, S0, q, k, v, beta, np.repeat(alpha[..., None], 128, -1))
+    np.testing.assert_array_equal(og, ok)
+    np.testing.assert_array_equal(Sg, Sk)
+
+
+def test_rank_grows_by_at_most_one_per_token(oracle_lib):
+    rng = np.random.default_rng(5)
+    dk = dv = 16
+    p = oracle.Params(dk=dk, dv=dv, bits=32, num_comp=0)
+    T = 6
+    q = np.stack([_unit(rng, dk) for _ in range(T)])[:, None].astype(np.float32)
+    k = np.stack([_unit(rng, dk) for _ in range(T)])[:, None].astype(np.float32)
+    v = rng.normal(size=(T, 1, dv)).astype(np.float32)
+    beta = rng.uniform(0.2, 0.9, (T, 1)).astype(np.float32)
+    a = rng.uniform(0.8, 1.0, (T, 1)).astype(np.float32)
+    for t in range(1, T + 1):
+        _, S, _ = oracle.run(p, np.zeros((1, dk, dv), np.float32), q[:t], k[:t], v[:t],
+                             beta[:t], a[:t])
+        assert np.linalg.matrix_rank(S[0], tol=1e-9) == t
+
+
+# --------------------------------------------------------------------------
+# per-window buffering is exact algebra
+
+@pytest.mark.parametrize("kda", [False, True])
+def test_buffered_window_equals_dense_recurrence(oracle_lib, kda):
+    """With no quantization inside the window, outputs computed from the
+    window-start state plus the buffered rank-one updates equal the
+    step-by-step recurrence (per-window paragraph; abstract)."""
+    rng = np.random.default_rng(6 + kda)
+    dk, dv, T = 32, 24, 16
+    S = _rand_state(rng, dk, dv, rows=(3,), cols=(5,))
+    q = np.stack([_unit(rng, dk) for _ in range(T)])
+    k = np.stack([_unit(rng, dk) for _ in range(T)])
+    v = rng.normal(size=(T, dv))
+    beta = rng.uniform(0.1, 0.9, T)
+    a = rng.uniform(0.5, 1.0, (T, dk)) if kda else np.repeat(rng.uniform(0.5, 1.0, (T, 1)), dk, 1)
+    ob, Sb = oracle.window_buffered(S, q, k, v, beta, a)
+    Sd = S.copy()
+    od = []
+    for t in range(T):
+        Sd, o, _ = oracle.step(Sd, q[t], k[t], v[t], beta[t], a[t])
+        od.append(o)
+    od = np.array(od)
+    assert np.linalg.norm(ob - od) <= 1e-12 * np.linalg.norm(od)
+    assert np.linalg.norm(Sb - Sd) <= 1e-12 * np.linalg.norm(Sd)
+
+
+def test_window_one_is_per_step_quantization(oracle_lib):
+    """W = 1 reduces to quantizing after every token."""
+    from linear_attention_recurrent_lq_b200 import inputs
+    wl = inputs.WORKLOADS["gdn_int8_b1h1"].replace(tokens=8, window=1)
+    d = inputs.draw(wl)
+    p = oracle.Params.of(wl)
+    o_run, S_run, _ = oracle.run(p, d["S0"].reshape(1, 128, 128), d["q"].reshape(8, 1, 128),
+                                 d["k"].reshape(8, 1, 128), d["v"].reshape(8, 1, 128),
+                                 d["beta"].reshape(8, 1), d["decay"].reshape(8, 1))
+
+    def requant(S):
+        c = oracle.compress(p, S.astype(np.float32))
+        return oracle.dequant(p, c["codes"], c["qs"], c["sm"], c["meta"], c["vec"])
+
+    S = requant(d["S0"][0, 0])
+    for t in range(8):
+        S, o, _ = oracle.step(S, d["q"][t, 0, 0], d["k"][t, 0, 0], d["v"][t, 0, 0],
+                              d["beta"][t, 0, 0], np.full(128, d["decay"][t, 0, 0], np.float64))
+        np.testing.assert_array_equal(o, o_run[t, 0])
+        S = requant(S)
+    np.testing.assert_array_equal(S, S_run[0])
+
+
+def test_partial_window_stays_unquantized(oracle_lib):
+    """Tokens after the last boundary are not requantized: running 20 tokens
+    with W = 16 equals 16 quantized tokens followed by 4 dense steps."""
+    from linear_attention_recurrent_lq_b200 import inputs
+    wl = inputs.WORKLOADS["gdn_int8_b1h1"].replace(tokens=20)
+    d = inputs.draw(wl)
+    p = oracle.Params.of(wl)
+    args = lambda n: (d["q"][:n].reshape(n, 1, 128), d["k"][:n].reshape(n, 1, 128),
+                      d["v"][:n].reshape(n, 1, 128), d["beta"][:n].reshape(n, 1),
+                      d["decay"][:n].reshape(n, 1))
+    _, S16, _ = oracle.run(p, d["S0"].reshape(1, 128, 128), *args(16))
+    o20, S20, _ = oracle.run(p, d["S0"].reshape(1, 128, 128), *args(20))
+    S = S16[0]
+    for t in range(16, 20):
+        S, o, _ = oracle.step(S, d["q"][t, 0, 0], d["k"][t, 0, 0], d["v"][t, 0, 0],
+                              d["beta"][t, 0, 0], np.full(128, d["decay"][t, 0, 0], np.float64))
+        np.testing.assert_array_equal(o, o20[t, 0])
+    np.testing.assert_array_equal(S, S20[0])
+
+
+# --------------------------------------------------------------------------
+# compress: compensators, smoothing, quantization
+
+def _params(dk, dv, bits=8, r=4, smoothing=True, f16=False):
+    return oracle.Params(dk=dk, dv=dv, bits=bits, num_comp=r, smoothing=smoothing, scale_f16=f16)
+
+
+@pytest.mark.parametrize("bits", [8, 6, 4])
+def test_compensators_plus_residual_reconstruct_state_exactly(oracle_lib, bits):
+    rng = np.random.default_rng(10 + bits)
+    dk, dv = 32, 48
+    S = _rand_state(rng, dk, dv, rows=(1, 7), cols=(4, 40)).astype(np.float32)
+    p = _params(dk, dv, bits=bits, r=5)
+    c = oracle.compress(p, S)
+    rebuilt = c["R"].copy()
+    lines = set()
+    for m, w in zip(c["meta"][:c["ncomp"]], c["vec"]):
+        assert m not in lines
+        lines.add(int(m))
+        if m & oracle.KIND_COL:
+            j = m & 0x7FFFFFFF
+            assert np.all(c["R"][:, j] == 0)
+            rebuilt[:, j] += w[:dk]
+        else:
+            assert np.all(c["R"][m] == 0)
+            rebuilt[m] += w[:dv]
+    np.testing.assert_array_equal(rebuilt, S.astype(np.float64))
+    # the planted outlier lines are the ones taken
+    assert {1, 7, oracle.KIND_COL | 4, oracle.KIND_COL | 40} <= lines
+
+
+def test_greedy_choice_matches_brute_force(oracle_lib):
+    rng = np.random.default_rng(20)
+    for trial in range(40):
+        dk, dv = rng.choice([2, 4, 8]), rng.choice([2, 4, 8])
+        S = rng.normal(size=(dk, dv)).astype(np.float32)
+        if trial % 3 == 0:      # exact ties between a row and a column
+            S = np.round(S * 2) / 2
+            S[:, 0] = 0
+            S[0, :] = 0
+            S[0, 0] = 2.0
+        r = int(rng.integers(1, min(dk, dv) + 1))
+        p = _params(dk, dv, bits=8, r=r, smoothing=bool(trial % 2))
+        c = oracle.compress(p, S)
+        b = brute.compress(S, 8, r, bool(trial % 2))
+        assert list(c["meta"][:c["ncomp"]]) == b["meta"]
+        np.testing.assert_array_equal(c["sm"], b["sm"])
+        np.testing.assert_array_equal(c["qs"], b["qs"])
+        np.testing.assert_array_equal(c["codes"], b["codes"])
+
+
+@pytest.mark.parametrize("name", ["compress_ties.json"])
+def test_golden_tie_order(oracle_lib, name):
+    g = json.load(open(os.path.join(GOLDEN, name)))
+    for case in g["cases"]:
+        S = np.array(case["S"], np.float32)
+        p = _params(S.shape[0], S.shape[1], bits=8, r=case["num_comp"])
+        c = oracle.compress(p, S)
+        assert [int(x) for x in c["meta"]] == case["meta"]
+
+
+@pytest.mark.parametrize("name", ["compress_4x4_int4.json", "compress_fp32_quotient.json"])
+def test_golden_compress(oracle_lib, name):
+    g = json.load(open(os.path.join(GOLDEN, name)))
+    pr = g["params"]
+    p = oracle.Params(dk=pr["dk"], dv=pr["dv"], bits=pr["bits"], num_comp=pr["num_comp"],
+                      smoothing=pr["smoothing"], scale_f16=pr["scale_f16"])
+    c = oracle.compress(p, np.array(g["S"], np.float32))
+    if "meta" in g:
+        assert [int(x) for x in c["meta"]] == g["meta"]
+        np.testing.assert_array_equal(c["vec"], np.array(g["vec"], np.float32))
+    if "sm" in g:
+        np.testing.assert_array_equal(c["sm"], np.array(g["sm"], np.float32))
+    np.testing.assert_array_equal(c["qs"], np.array(g["qs"], np.float32))
+    np.testing.assert_array_equal(c["codes"], np.array(g["codes_value_major"], np.int8))
+
+
+@pytest.mark.parametrize("f16", [False, True])
+def test_smoothing_is_power_of_two_and_exactly_invertible(oracle_lib, f16):
+    rng = np.random.default_rng(30)
+    dk, dv = 64, 64
+    S = _rand_state(rng, dk, dv, rows=(2, 9), cols=(11,), gain=100.0).astype(np.float32)
+    S[5] = 0.0          # an all-zero key row
+    S[6] *= 1e-3        # a tiny one
+    p = _params(dk, dv, bits=8, r=2, f16=f16)
+    c = oracle.compress(p, S)
+    R = c["R"].astype(np.float32)
+    sm = c["sm"]
+    mant, _ = np.frexp(sm)
+    assert np.all(mant == 0.5), "smoothing scales must be powers of two"
+    Rs = R / sm[:, None]
+    np.testing.assert_array_equal(Rs * sm[:, None], R)
+    rowmax = np.abs(Rs).max(axis=1)
+    nz = np.abs(R).max(axis=1) > 0
+    assert np.all((rowmax[nz] > 0.5) & (rowmax[nz] <= 1.0))
+    assert np.all(sm[~nz] == 1.0)
+    p0 = _params(dk, dv, bits=8, r=2, smoothing=False, f16=f16)
+    assert np.all(oracle.compress(p0, S)["sm"] == 1.0)
+
+
+@pytest.mark.parametrize("bits,f16,smoothing", [(8, False, True), (8, False, False),
+                                                 (6, True, True), (4, True, True)])
+def test_quantization_error_bound(oracle_lib, bits, f16, smoothing):
+    """Symmetric rounding per value column of the smoothed residual: every
+    entry off a compensated line is within half a step sm_i*qs_j/2, entries on
+    compensated lines are exact, and each nonzero column reaches Qmax."""
+    rng = np.random.default_rng(40 + bits)
+    dk, dv = 64, 32
+    S = _rand_state(rng, dk, dv, rows=(0, 13), cols=(7,), gain=80.0).astype(np.float32)
+    p = _params(dk, dv, bits=bits, r=3, smoothing=smoothing, f16=f16)
+    c = oracle.compress(p, S)
+    D = oracle.dequant(p, c["codes"], c["qs"], c["sm"], c["meta"], c["vec"])
+    err = np.abs(D - S.astype(np.float64))
+    bound = 0.5 * c["sm"].astype(np.float64)[:, None] * c["qs"].astype(np.float64)[None, :]
+    comp_rows = [int(m) for m in c["meta"] if m != oracle.NONE and not m & oracle.KIND_COL]
+    comp_cols = [int(m & 0x7FFFFFFF) for m in c["meta"] if m != oracle.NONE and m & oracle.KIND_COL]
+    mask = np.ones_like(err, bool)
+    mask[comp_rows, :] = False
+    mask[:, comp_cols] = False
+    # the stored scale is rounded, so allow its relative rounding on top
+    slack = 2.0 ** -10 if f16 else 2.0 ** -22
+    assert np.all(err[mask] <= bound[mask] * (1 + slack) + 1e-30)
+    assert np.all(err[~mask] == 0)
+    assert np.abs(c["codes"]).max() <= p.qmax
+    colmax = np.abs(c["codes"].astype(int)).max(axis=1)
+    live = c["qs"] > 0
+    assert np.all(colmax[live] >= p.qmax - (1 if f16 else 0))
+
+
+def test_f16_scale_rounding_matches_numpy(oracle_lib):
+    rng = np.random.default_rng(50)
+    xs = np.concatenate([rng.uniform(-1, 1, 2000) * 10.0 ** rng.integers(-9, 5, 2000),
+                         [2 ** -24, 2 ** -25, 3 * 2 ** -26, 65504.0, 65519.0, 1.0 + 2 ** -11,
+                          1.0 + 3 * 2 ** -11, 2 ** -14 * (1 + 2 ** -10)]]).astype(np.float32)
+    for x in xs:
+        assert oracle.round_f16(float(x)) == float(np.float16(x)), x
+
+
+def test_pack_unpack_round_trip(oracle_lib):
+    rng = np.random.default_rng(60)
+    for bits in (8, 6, 4):
+        q = 2 ** (bits - 1)
+        codes = rng.integers(-q, q, size=(9, 128)).astype(np.int8)
+        packed = oracle.pack_rows(bits, codes)
+        assert packed.shape == (9, 128 * bits // 8)
+        np.testing.assert_array_equal(oracle.unpack_rows(bits, packed, 128), codes)
+
+
+def test_golden_packed_rows(oracle_lib):
+    g = json.load(open(os.path.join(GOLDEN, "packed_rows.json")))
+    for key, bits in (("int4", 4), ("int6", 6)):
+        codes = np.array([g[key]["codes"]], np.int8)
+        packed = oracle.pack_rows(bits, codes)
+        assert packed.tobytes().hex() == g[key]["bytes_hex"]
+        np.testing.assert_array_equal(oracle.unpack_rows(bits, packed, 16), codes)
+
+
+# --------------------------------------------------------------------------
+# whole sequences
+
+def test_run_matches_brute_force_on_tiny_heads(oracle_lib):
+    rng = np.random.default_rng(70)
+    for kda, bits, smoothing in ((False, 8, True), (True, 4, True), (False, 6, False)):
+        dk = dv = 16
+        T, W, r = 13, 4, 2
+        S0 = _rand_state(rng, dk, dv, rows=(2,), cols=(9,), gain=20.0).astype(np.float32)
+        q = np.stack([_unit(rng, dk) for _ in range(T)]).astype(np.float32)
+        k = np.stack([_unit(rng, dk) for _ in range(T)]).astype(np.float32)
+        v = rng.normal(size=(T, dv)).astype(np.float32)
+        beta = rng.uniform(0.1, 0.9, T).astype(np.float32)
+        a = (rng.uniform(0.6, 1.0, (T, dk)) if kda else
+             np.repeat(rng.uniform(0.6, 1.0, (T, 1)), dk, 1)).astype(np.float32)
+        p = oracle.Params(dk=dk, dv=dv, window=W, num_comp=r, bits=bits, kda=kda,
+                          smoothing=smoothing)
+        dec = a[:, None, :] if kda else a[:, :1]
+        o, S, _ = oracle.run(p, S0[None], q[:, None], k[:, None], v[:, None], beta[:, None], dec)
+        ob, Sb = brute.run(S0, q, k, v, beta, a, W, bits, r, smoothing)
+        np.testing.assert_allclose(o[:, 0], ob, rtol=1e-9, atol=1e-12)
+        np.testing.assert_allclose(S[0], Sb, rtol=1e-9, atol=1e-12)
+
+
+def _err_vs_fp32(wl, **kw):
+    from linear_attention_recurrent_lq_b200 import inputs
+    d = inputs.draw(wl)
+    T = wl.tokens
+    args = (d["S0"].reshape(1, 128, 128), d["q"].reshape(T, 1, 128), d["k"].reshape(T, 1, 128),
+            d["v"].reshape(T, 1, 128), d["beta"].reshape(T, 1), d["decay"].reshape(T, 1))
+    p = oracle.Params.of(wl)
+    o_ref, _, _ = oracle.run(oracle.Params(**{**p.__dict__, "bits": 32}), *args)
+    o, _, _ = oracle.run(oracle.Params(**{**p.__dict__, **kw}), *args)
+    return np.linalg.norm(o - o_ref) / np.linalg.norm(o_ref)
+
+
+def test_window_quantization_accumulates_less_error_than_per_step(oracle_lib):
+    """Per-window paragraph: quantizing once per window instead of every
+    token keeps rounding error from compounding."""
+    from linear_attention_recurrent_lq_b200 import inputs
+    wl = inputs.WORKLOADS["gdn_int8_b1h1"].replace(tokens=64, bits=6, smoothing=True)
+    e_step = _err_vs_fp32(wl, window=1)
+    e_win = _err_vs_fp32(wl, window=16)
+    assert e_win < 0.5 * e_step, (e_win, e_step)
+
+
+def test_compensators_and_smoothing_reduce_error(oracle_lib):
+    """Compensator Tokens paragraph: taking the outlier lines out as FP32
+    pairs lowers the quantization error.  Residual smoothing paragraph: when
+    the residual's key rows are still uneven, balancing them before
+    quantizing lowers it further.  More bits lower it too."""
+    from linear_attention_recurrent_lq_b200 import inputs
+    wl = inputs.WORKLOADS["gdn_int8_b1h1"].replace(tokens=32, bits=6)
+    plain = _err_vs_fp32(wl, num_comp=0, smoothing=False)
+    comp = _err_vs_fp32(wl, num_comp=3, smoothing=False)
+    assert comp < 0.1 * plain, (plain, comp)
+    # one compensator for three outlier lines leaves uneven key rows behind
+    assert _err_vs_fp32(wl, num_comp=1, smoothing=True) < 0.5 * _err_vs_fp32(
+        wl, num_comp=1, smoothing=False)
+    graded = wl.replace(outlier_rows=6, row_gain=8.0, outlier_cols=0)
+    assert _err_vs_fp32(graded, num_comp=1, smoothing=True) < 0.7 * _err_vs_fp32(
+        graded, num_comp=1, smoothing=False)
+    e = [_err_vs_fp32(wl, bits=b, num_comp=3, smoothing=True) for b in (8, 6, 4)]
+    assert e[0] < e[1] < e[2], e
