@@ -1,0 +1,548 @@
+#!/usr/bin/env python
+"""Decode throughput of the LeapQuant low-bit recurrent state on B200.
+
+Metric: decode head-tokens/s (one head-token = one (sequence, head) state
+advanced by one generated token) and the achieved HBM bandwidth of the decode
+kernel against the measured copy bandwidth, next to the library's own
+FP32-state kernel on the same inputs.
+
+Workload (default gdn_int8_b64h32): Gated DeltaNet heads, batch 64 x 32 heads,
+dk = dv = 128, INT8 state with smoothing, W = 16, r = 4 compensators, bf16
+q/k/v.  One step = one window: W decode tokens over L layer-states (each its
+own 64 x 32 heads, as consecutive linear-attention layers of a model), then
+the L window flushes.  Rotating L = 8 layers keeps the working set (~0.6 GB of
+state) well above the 126 MB L2, so every token re-reads its state from HBM;
+no L2 flush is needed.  Inputs are seeded synthetic draws, resident in HBM
+before timing; every step reuses the same window of inputs on an evolving
+state.
+
+Launch: python bench.py [--gpus N --steps K --warmup W]; for N > 1 under
+torch.distributed.run, one process per GPU, each rank advancing its own
+replica of the workload (independent sequences: no collective on the data
+path), timed as the max over ranks.  --impl reference times the CPU oracle
+(the FP64 restatement of the method) on a bounded sample instead.
+"""
+from __future__ import annotations
+
+import argparse
+import hashlib
+import json
+import math
+import os
+import statistics
+import subprocess
+import sys
+import time
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+
+def parse_args():
+    ap = argparse.ArgumentParser(description=__doc__.split("\n\n")[0])
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=600)
+    ap.add_argument("--warmup", type=int, default=10)
+    ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
+    ap.add_argument("--workload", default="gdn_int8_b64h32")
+    ap.add_argument("--layers", type=int, default=8)
+    ap.add_argument("--fp32-steps", type=int, default=0, help="0: steps/4")
+    ap.add_argument("--e2e-steps", type=int, default=0, help="0: steps/10")
+    ap.add_argument("--no-e2e", action="store_true")
+    ap.add_argument("--no-fp32", action="store_true")
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--cpu-seconds", type=float, default=10.0)
+    return ap.parse_args()
+
+
+# ------------------------------------------------------------ byte model
+
+def field_bytes(wl):
+    """Bytes of every blob field and input, per head (no padding)."""
+    dk, dv, r = wl.dk, wl.dv, wl.num_comp
+    sb = 2 if wl.scale_dtype == "f16" else 4
+    ib = 2 if wl.in_dtype == "bf16" else 4
+    kda = wl.decay_kind == "kda"
+    return dict(
+        hdr=20, meta=4 * r, qs=sb * dv, sm=sb * dk, cvec=4 * r * max(dk, dv),
+        codes=dv * dk * wl.bits // 8, pair=4 * (dk + dv), g=4 * dk if kda else 0,
+        inputs=ib * (2 * dk + dv) + 4 + (4 * dk if kda else 4), out=4 * dv)
+
+
+def decode_bytes(wl, count):
+    """Algorithmic bytes one decode step moves for one head with `count`
+    pairs already buffered: it reads the header, scales, compensators, codes,
+    the buffered pairs, the decay product and the token's inputs, and writes
+    the output, the new pair, the decay product and the count."""
+    f = field_bytes(wl)
+    read = (f["hdr"] + f["meta"] + f["qs"] + f["sm"] + f["cvec"] + f["codes"] + count * f["pair"]
+            + f["g"] + f["inputs"])
+    write = f["out"] + f["pair"] + f["g"] + 8
+    return read + write
+
+
+def flush_bytes(wl):
+    """Algorithmic bytes of one window flush per head: read the compact state,
+    W pairs and the decay product; write the new compact state and header."""
+    f = field_bytes(wl)
+    compact = f["qs"] + f["sm"] + f["cvec"] + f["codes"]
+    return (f["hdr"] + f["meta"] + compact + wl.window * f["pair"] + f["g"]) + \
+           (compact + f["meta"] + 16 + f["g"])
+
+
+def fp32_bytes(wl):
+    """FP32-state step per head: read and write the dense state, read inputs,
+    write the output."""
+    f = field_bytes(wl)
+    return 2 * 4 * wl.dk * wl.dv + f["inputs"] + f["out"]
+
+
+# ------------------------------------------------------------ helpers
+
+def kernel_source_sha():
+    h = hashlib.sha256()
+    paths = sorted(os.path.join(ROOT, "linear_attention_recurrent_lq_b200", "csrc", n)
+                   for n in os.listdir(os.path.join(ROOT, "linear_attention_recurrent_lq_b200", "csrc")))
+    for p in paths + [os.path.join(ROOT, "include", "leapquant.h")]:
+        with open(p, "rb") as fh:
+            h.update(fh.read())
+    return h.hexdigest()[:16]
+
+
+def profiled_traffic(name):
+    """DRAM bytes per launch from the committed ncu summary, if it was taken
+    on the current kernel sources; else None."""
+    path = os.path.join(ROOT, "profiles", name)
+    if not os.path.exists(path):
+        return None
+    vals = {}
+    for line in open(path):
+        if ":" in line and line.strip().startswith(("traffic_bytes_per_launch", "kernel_source_sha")):
+            k, v = line.split(":", 1)
+            vals[k.strip()] = v.strip().strip("`")
+    if vals.get("kernel_source_sha") != kernel_source_sha():
+        return None
+    try:
+        return int(float(vals["traffic_bytes_per_launch"]))
+    except (KeyError, ValueError):
+        return None
+
+
+def measured_peaks():
+    path = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    if os.path.exists(path):
+        with open(path) as fh:
+            return json.load(fh), "measured"
+    return {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0}, "fallback"
+
+
+class Clocks:
+    """nvidia-smi samples of one GPU while the timed region runs."""
+
+    FIELDS = ("index,uuid,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+              "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
+              "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, uuid):
+        self.uuid = uuid
+        self.proc = None
+
+    def start(self):
+        try:
+            self.proc = subprocess.Popen(
+                ["nvidia-smi", "--query-gpu=" + self.FIELDS, "--format=csv,noheader,nounits",
+                 "-lms", "100"], stdout=subprocess.PIPE, stderr=subprocess.DEVNULL, text=True)
+        except OSError:
+            self.proc = None
+        time.sleep(0.3)
+
+    def stop(self):
+        if self.proc is None:
+            return None
+        time.sleep(0.2)
+        self.proc.terminate()
+        try:
+            out, _ = self.proc.communicate(timeout=5)
+        except subprocess.TimeoutExpired:
+            self.proc.kill()
+            out, _ = self.proc.communicate()
+        rows = []
+        for line in out.splitlines():
+            parts = [x.strip() for x in line.split(",")]
+            if len(parts) < 10:
+                continue
+            if self.uuid and self.uuid not in parts[1]:
+                continue
+            rows.append(parts)
+        if not rows:
+            return None
+        sm = [float(r[2]) for r in rows if r[2].replace(".", "").isdigit()]
+        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        reasons = sorted({names[i] for r in rows for i in range(4) if r[6 + i].lower() == "active"})
+        return {"sm_mhz": statistics.median(sm) if sm else None,
+                "sm_max_mhz": float(rows[0][3]) if rows[0][3].replace(".", "").isdigit() else None,
+                "reasons": reasons, "samples": len(rows),
+                "power_w_max": max(float(r[4]) for r in rows
+                                   if r[4].replace(".", "").isdigit()) if rows else None}
+
+
+def dist_setup():
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    return world, rank, local
+
+
+# ------------------------------------------------------------ our arm
+
+class Arm:
+    """L layer-states of one workload on this GPU, with captured graphs."""
+
+    def __init__(self, wl, layers_data, bits, torch, B):
+        self.wl, self.torch, self.B = wl, torch, B
+        self.cfg = B.config_for(wl, bits=bits)
+        self.bits = bits
+        self.L = len(layers_data)
+        self.states, self.inp, self.out = [], [], []
+        for ld in layers_data:
+            st = B.LQState(self.cfg)
+            st.init(ld["S0"])
+            self.states.append(st)
+            self.inp.append(ld["dev"])
+            self.out.append(torch.empty((wl.window, wl.batch, wl.heads, wl.dv), dtype=torch.float32,
+                                        device="cuda"))
+        torch.cuda.synchronize()
+
+    def decode_all(self):
+        W = self.wl.window
+        for t in range(W):
+            for l in range(self.L):
+                x = self.inp[l]
+                self.states[l].step(x["q"][t], x["k"][t], x["v"][t], x["beta"][t], x["decay"][t],
+                                    self.out[l][t])
+
+    def flush_all(self):
+        if self.bits == 32:
+            return
+        for l in range(self.L):
+            self.states[l].flush()
+
+    def capture(self):
+        torch = self.torch
+        # one eager window first: sets kernel attributes outside capture
+        self.decode_all()
+        self.flush_all()
+        torch.cuda.synchronize()
+        s = torch.cuda.Stream()
+        s.wait_stream(torch.cuda.current_stream())
+        self.g_dec, self.g_fl = torch.cuda.CUDAGraph(), torch.cuda.CUDAGraph()
+        with torch.cuda.graph(self.g_dec, stream=s):
+            self.decode_all()
+        if self.bits != 32:
+            with torch.cuda.graph(self.g_fl, stream=s):
+                self.flush_all()
+        torch.cuda.synchronize()
+
+    def step(self):
+        self.g_dec.replay()
+        if self.bits != 32:
+            self.g_fl.replay()
+
+    def launches_per_step(self):
+        return self.wl.window * self.L + (self.L if self.bits != 32 else 0)
+
+
+def time_arm(arm, steps, warmup, torch, dist, world):
+    """Time `steps` window-steps; returns total ms (max over ranks) and the
+    per-step decode / flush split from events recorded between the graphs."""
+    for _ in range(warmup):
+        arm.step()
+    torch.cuda.synchronize()
+    E = torch.cuda.Event
+    marks = [(E(enable_timing=True), E(enable_timing=True), E(enable_timing=True)) for _ in range(steps)]
+    start, end = E(enable_timing=True), E(enable_timing=True)
+    if world > 1:
+        dist.barrier()
+    torch.cuda.synchronize()
+    start.record()
+    for s in range(steps):
+        a, b, c = marks[s]
+        a.record()
+        arm.g_dec.replay()
+        b.record()
+        if arm.bits != 32:
+            arm.g_fl.replay()
+        c.record()
+    end.record()
+    torch.cuda.synchronize()
+    if world > 1:
+        dist.barrier()
+    total = start.elapsed_time(end)
+    dec = sum(a.elapsed_time(b) for a, b, _ in marks)
+    fl = sum(b.elapsed_time(c) for _, b, c in marks)
+    if world > 1:
+        t = torch.tensor([total, dec, fl], device="cuda", dtype=torch.float64)
+        dist.all_reduce(t, op=dist.ReduceOp.MAX)
+        total, dec, fl = t.tolist()
+    return total, dec, fl
+
+
+def time_e2e(arm, host, steps, torch, dist, world):
+    """Same steps through the public calls with host buffers: every step
+    copies its inputs host->device from pinned memory, runs the window and
+    copies every output back."""
+    h2d = sum(t.numel() * t.element_size() for ld in host for t in ld["in"].values())
+    d2h = sum(o.numel() * o.element_size() for o in arm.out)
+
+    def one():
+        for l, ld in enumerate(host):
+            for name, t in ld["in"].items():
+                arm.inp[l][name].copy_(t, non_blocking=True)
+        arm.step()
+        for l, ld in enumerate(host):
+            ld["out"].copy_(arm.out[l], non_blocking=True)
+
+    one()
+    torch.cuda.synchronize()
+    E = torch.cuda.Event
+    start, end = E(enable_timing=True), E(enable_timing=True)
+    if world > 1:
+        dist.barrier()
+    torch.cuda.synchronize()
+    start.record()
+    for _ in range(steps):
+        one()
+    end.record()
+    torch.cuda.synchronize()
+    if world > 1:
+        dist.barrier()
+    ms = start.elapsed_time(end)
+    if world > 1:
+        t = torch.tensor([ms], device="cuda", dtype=torch.float64)
+        dist.all_reduce(t, op=dist.ReduceOp.MAX)
+        ms = t.item()
+    return ms, h2d, d2h
+
+
+def make_layers(wl, L, torch, I):
+    layers = []
+    for l in range(L):
+        s = I.InputStream(wl, stream=l)
+        st = s.state()
+        tk = s.tokens(wl.window)
+        d = {**st, **tk}
+        layers.append({"S0": torch.from_numpy(st["S0"]).cuda(), "dev": I.to_device(wl, d), "np": d})
+    return layers
+
+
+def cpu_baseline(wl, layer_np, seconds, oracle):
+    """The oracle as it stands on this host's cores, on a sample of the same
+    workload: heads of layer 0, its window of tokens repeated, sized to run
+    for about `seconds`."""
+    import numpy as np
+    p = oracle.Params.of(wl)
+    nh = wl.batch * wl.heads
+    W = wl.window
+
+    def run(nheads, nwin):
+        heads = np.arange(nheads)
+        T = W * nwin
+        tile = lambda x: np.tile(x, (nwin,) + (1,) * (x.ndim - 1))
+        S0 = layer_np["S0"].reshape(nh, wl.dk, wl.dv)[heads]
+        q = tile(layer_np["q"].reshape(W, nh, wl.dk)[:, heads])
+        k = tile(layer_np["k"].reshape(W, nh, wl.dk)[:, heads])
+        v = tile(layer_np["v"].reshape(W, nh, wl.dv)[:, heads])
+        beta = tile(layer_np["beta"].reshape(W, nh)[:, heads])
+        dshape = (W, nh, wl.dk) if wl.decay_kind == "kda" else (W, nh)
+        decay = tile(layer_np["decay"].reshape(dshape)[:, heads])
+        t0 = time.perf_counter()
+        _, _, used = oracle.run(p, S0, q, k, v, beta, decay, threads=0)
+        return time.perf_counter() - t0, used, nheads * T
+
+    dt, used, n = run(min(nh, 64), 1)
+    rate = n / dt
+    nheads = min(nh, max(1, int(rate * seconds / W)))
+    nwin = max(1, int(round(rate * seconds / (nheads * W))))
+    nwin = min(nwin, 64)
+    dt, used, n = run(nheads, nwin)
+    return {"value": n / dt, "unit": "head-tokens/s", "cores": used, "kind": "oracle",
+            "sample": f"{nheads} heads of one layer x {W * nwin} tokens (its first window of "
+                      f"{W} tokens repeated {nwin}x), FP64 C oracle, OpenMP over heads, "
+                      f"{dt:.1f} s"}
+
+
+def config_of(wl, args, world):
+    return {"workload": wl.name, "batch": wl.batch, "heads": wl.heads, "dk": wl.dk, "dv": wl.dv,
+            "window": wl.window, "num_comp": wl.num_comp, "state_bits": wl.bits,
+            "decay": wl.decay_kind, "smoothing": wl.smoothing, "scales": wl.scale_dtype,
+            "qkv_dtype": wl.in_dtype, "layers_rotated": args.layers,
+            "step": f"one window: {wl.window} decode tokens x {args.layers} layers + {args.layers} flushes",
+            "l2": "no flush: the rotated layer-states are larger than L2",
+            "parallelism": f"replicas x{world}" if world > 1 else "single GPU"}
+
+
+def main_ours(args):
+    import numpy as np
+    import torch
+    world, rank, local = dist_setup()
+    dist = None
+    if world > 1:
+        import datetime
+        import torch.distributed as dist
+        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=300))
+    torch.cuda.set_device(local)
+    import __graft_entry__
+    __graft_entry__.build()
+    from linear_attention_recurrent_lq_b200 import binding as B
+    from linear_attention_recurrent_lq_b200 import inputs as I
+
+    wl = I.WORKLOADS[args.workload]
+    if rank:
+        wl = wl.replace(seed=wl.seed + 1000 * rank)  # other sequences on other ranks
+    L = args.layers
+    layers = make_layers(wl, L, torch, I)
+    peaks, peak_kind = measured_peaks()
+    hbm = float(peaks["hbm_gbs"])
+    nh = wl.batch * wl.heads
+
+    # ---- LeapQuant arm
+    arm = Arm(wl, layers, wl.bits, torch, B)
+    arm.capture()
+    props = torch.cuda.get_device_properties(local)
+    uuid = str(getattr(props, "uuid", "") or "")
+    clocks = Clocks(uuid)
+    clocks.start()
+    total, dec, fl = time_arm(arm, args.steps, args.warmup, torch, dist, world)
+    clk = clocks.stop()
+    status = max(st.check() for st in arm.states)
+    if status != 0:
+        raise RuntimeError(f"device status after timing: {B.STATUS_NAMES[status]}")
+    W = wl.window
+    head_tokens = args.steps * W * L * nh * world
+    value = head_tokens / (total / 1e3)
+    dec_launches = args.steps * W * L
+    dec_bytes_per_launch = nh * sum(decode_bytes(wl, c) for c in range(W)) / W
+    dec_ms = dec / dec_launches
+    achieved = dec_bytes_per_launch / (dec_ms / 1e3) / 1e9
+    traffic = profiled_traffic(f"decode_{wl.name}.md")
+    fl_launches = args.steps * L
+    fl_ms = fl / fl_launches
+    step_bytes = nh * L * (sum(decode_bytes(wl, c) for c in range(W)) + flush_bytes(wl))
+    line = {
+        "metric": "decode head-tokens/s and achieved HBM GB/s (% of B200 peak) vs FP32-state kernel",
+        "value": value, "unit": "head-tokens/s", "n_gpus": world, "steps": args.steps,
+        "warmup": args.warmup, "ms_per_step": total / args.steps, "higher_is_better": True,
+        "scaling": "weak", "vs_baseline": None, "dtype": "f32", "data": "synthetic",
+        "config": config_of(wl, args, world),
+        "roofline": {"bound": "hbm", "achieved": achieved, "peak": hbm, "unit": "GB/s",
+                     "frac": achieved / hbm, "traffic": traffic,
+                     "kernel": "decode_kernel<128,8>", "peak_source": f"{peak_kind} hbm_gbs",
+                     "algorithmic_bytes_per_launch": dec_bytes_per_launch,
+                     "avg_launch_us": dec_ms * 1e3},
+        "step_hbm": {"algorithmic_bytes_per_step": step_bytes,
+                     "achieved_gbs": step_bytes / (total / args.steps / 1e3) / 1e9 * world,
+                     "frac": step_bytes / (total / args.steps / 1e3) / 1e9 / hbm,
+                     "flush_avg_launch_us": fl_ms * 1e3,
+                     "flush_algorithmic_bytes_per_launch": nh * flush_bytes(wl)},
+        "gpu_launches": args.steps * arm.launches_per_step(),
+        "clocks": clk,
+    }
+
+    # ---- FP32-state kernel on the same inputs (the comparison point)
+    if not args.no_fp32:
+        arm32 = Arm(wl, layers, 32, torch, B)
+        arm32.capture()
+        ks = args.fp32_steps or max(4, args.steps // 4)
+        t32, d32, _ = time_arm(arm32, ks, max(3, args.warmup // 2), torch, dist, world)
+        v32 = ks * W * L * nh * world / (t32 / 1e3)
+        b32 = nh * fp32_bytes(wl)
+        a32 = b32 / (d32 / (ks * W * L) / 1e3) / 1e9
+        line["fp32_state"] = {"value": v32, "unit": "head-tokens/s", "steps": ks,
+                              "achieved_gbs": a32, "frac": a32 / hbm,
+                              "algorithmic_bytes_per_launch": b32}
+        line["vs_fp32_state_kernel"] = value / v32
+        del arm32
+        torch.cuda.empty_cache()
+
+    # ---- end to end through the public calls with host buffers
+    if not args.no_e2e:
+        host = []
+        for l in range(L):
+            hin = {k: v.cpu().pin_memory() for k, v in layers[l]["dev"].items()}
+            host.append({"in": hin, "out": torch.empty_like(arm.out[l], device="cpu").pin_memory()})
+        ke = args.e2e_steps or max(3, args.steps // 10)
+        ms, h2d, d2h = time_e2e(arm, host, ke, torch, dist, world)
+        line["e2e"] = {"value": ke * W * L * nh * world / (ms / 1e3), "unit": "head-tokens/s",
+                       "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h,
+                       "steps": ke, "ms_per_step": ms / ke}
+
+    if rank == 0 and world == 1 and not args.no_cpu_baseline:
+        import oracle
+        line["cpu_baseline"] = cpu_baseline(wl, layers[0]["np"], args.cpu_seconds, oracle)
+
+    if rank == 0:
+        print(json.dumps(line), flush=True)
+    if world > 1:
+        dist.barrier()
+        dist.destroy_process_group()
+
+
+def main_reference(args):
+    """The oracle, as it stands, timed on the host cores on bounded samples of
+    the same workload (rank 0 only)."""
+    world, rank, _ = dist_setup()
+    if rank != 0:
+        return
+    sys.path.insert(0, ROOT)
+    import numpy as np
+    import oracle
+    from oracle import build as ob
+    from linear_attention_recurrent_lq_b200 import inputs as I
+    ob.build()
+    wl = I.WORKLOADS[args.workload]
+    s = I.InputStream(wl, stream=0)
+    ld = {**s.state(), **s.tokens(wl.window)}
+    p = oracle.Params.of(wl)
+    nh = wl.batch * wl.heads
+    W = wl.window
+
+    def sample(nheads, h0):
+        heads = (np.arange(nheads) + h0) % nh
+        dshape = (W, nh, wl.dk) if wl.decay_kind == "kda" else (W, nh)
+        return (ld["S0"].reshape(nh, wl.dk, wl.dv)[heads], ld["q"].reshape(W, nh, wl.dk)[:, heads],
+                ld["k"].reshape(W, nh, wl.dk)[:, heads], ld["v"].reshape(W, nh, wl.dv)[:, heads],
+                ld["beta"].reshape(W, nh)[:, heads], ld["decay"].reshape(dshape)[:, heads])
+
+    t0 = time.perf_counter()
+    _, _, used = oracle.run(p, *sample(64, 0))
+    rate = 64 * W / (time.perf_counter() - t0)
+    budget = 90.0 / max(1, args.steps + args.warmup)  # seconds per step
+    nheads = int(min(nh, max(1, rate * budget / W)))
+    for x in range(args.warmup):
+        oracle.run(p, *sample(nheads, x * nheads))
+    t0 = time.perf_counter()
+    for x in range(args.steps):
+        _, _, used = oracle.run(p, *sample(nheads, x * nheads))
+    dt = time.perf_counter() - t0
+    value = args.steps * nheads * W / dt
+    args.layers = 1
+    desc = (f"per step: {nheads} heads x {W} tokens (one window incl. its flush) of "
+            f"{wl.name}, FP64 C oracle, OpenMP over heads")
+    print(json.dumps({
+        "metric": "decode head-tokens/s and achieved HBM GB/s (% of B200 peak) vs FP32-state kernel",
+        "value": value, "unit": "head-tokens/s", "n_gpus": world, "steps": args.steps,
+        "warmup": args.warmup, "ms_per_step": dt / args.steps * 1e3, "higher_is_better": True,
+        "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": "synthetic",
+        "config": config_of(wl, args, 1), "impl": "reference",
+        "cpu_baseline": {"value": value, "unit": "head-tokens/s", "cores": used, "kind": "oracle",
+                         "sample": desc},
+        "e2e": {"value": value, "unit": "head-tokens/s", "h2d_bytes_per_step": 0,
+                "d2h_bytes_per_step": 0}}), flush=True)
+
+
+if __name__ == "__main__":
+    a = parse_args()
+    if a.impl == "reference":
+        main_reference(a)
+    else:
+        main_ours(a)

@@ -1,0 +1,178 @@
+/*
+ * leapquant.h -- C ABI of the B200 (sm_100a) LeapQuant decode library.
+ *
+ * LeapQuant keeps the recurrent state of Gated DeltaNet (GDN) and Kimi Delta
+ * Attention (KDA) heads in 8, 6 or 4 bits.  The state is requantized once per
+ * window of W tokens instead of after every token; inside a window the low-bit
+ * state is fixed, each token's delta-rule update is kept in FP32 as a rank-one
+ * pair, and outputs are computed from the fixed state plus those pairs.  The
+ * largest outlier lines of the state are kept aside in FP32 as rank-one
+ * compensator pairs, and the remaining residual is balanced per key row
+ * before it is quantized.
+ * Sources: news post "Linear attention has to move state every token it
+ * generates; LeapQuant compresses it to 8-bit without losing accuracy"
+ * (paragraphs on per-window quantization, Compensator Tokens and residual
+ * smoothing) and "LeapQuant: Efficient Linear Attention with Accurate
+ * Recurrent State Quantization" (original abstract).  The pages print no
+ * equations; the step used is the delta rule
+ *     S' = D_t S,  u_t = beta_t (v_t - S'^T k_t),  S_t = S' + k_t u_t^T,
+ *     o_t = S_t^T q_t,
+ * with D_t = alpha_t I (GDN) or diag(a_t) (KDA), S dk x dv, row i = key
+ * channel, column j = value channel.
+ *
+ * Conventions for every entry point:
+ *  - The caller allocates every buffer (device memory unless stated).  The
+ *    library allocates nothing and keeps no state between calls.
+ *  - Work is enqueued on `stream` and the call returns without waiting,
+ *    except lq_check_status, which synchronizes the stream.
+ *  - Argument errors are reported before anything is launched (LQ_ERR_*).
+ *    A failed launch returns LQ_ERR_CUDA.  Conditions that depend on data on
+ *    the device (a full window, a decay product out of range, a timed-out
+ *    wait) set a sticky bit in that (slot, head)'s status word; the kernels
+ *    then skip that (slot, head) and never trap.  lq_check_status reads them.
+ *  - Tensors are dense, row-major, contiguous.  N = num_slots (sequences),
+ *    H = num_heads.  The state buffer holds N*H consecutive blobs of
+ *    lq_state_bytes(cfg) bytes each, blob (n, h) at index n*H + h.  Pointers
+ *    must be 16-byte aligned and the state buffer 256-byte aligned
+ *    (LQ_ERR_MISALIGNED otherwise).
+ *  - Calls on one state must be ordered (same stream or explicit events);
+ *    calls on disjoint states may run concurrently.
+ *
+ * Per-(slot, head) blob layout (bits 8/6/4), offsets in bytes, every region
+ * 128-byte aligned, total rounded up to 256:
+ *    0    header: u32 count (tokens buffered in this window), u32 status
+ *         (device error bits), u32 ncomp (compensators in use), u32 magic,
+ *         f32 g (GDN: decay product since the window start), pad to 64,
+ *         u32 comp_meta[16] at 64 (bit 31: 1 = value column, 0 = key row;
+ *         bits 0..30: its index; 0xFFFFFFFF = unused)
+ *    128  KDA only: f32 g[dk], decay product per key channel since the
+ *         window start
+ *    then qs[dv]  quantization scale per value column (f32 or f16)
+ *    then sm[dk]  smoothing scale per key row, a power of two (f32 or f16)
+ *    then comp_vec[r][max(dk,dv)] f32: the compensator lines (a key row's
+ *         values over dv, or a value column's values over dk)
+ *    then codes[dv][dk*bits/8]: one row per value column, key index
+ *         ascending, groups of 16 codes:
+ *           8-bit: 16 bytes, byte b = code b, two's complement;
+ *           4-bit: 8 bytes, byte b = code 2b (low nibble) | code 2b+1 (high);
+ *           6-bit: 12 bytes = little-endian words w0,w1,w2: codes 4q..4q+3
+ *                  in bits 0..5 of the bytes of w_q; code 12+b split over
+ *                  bits 6..7 of byte b of w0 (its bits 0-1), w1 (2-3),
+ *                  w2 (4-5); 6-bit two's complement.
+ *    then pairs[W][dk+dv] f32: buffered pair m = khat_m (dk) then u_m (dv),
+ *         khat_m = k_m / g_m (the key in the window-start frame).
+ * The dense state the blob stands for is
+ *    S = diag(g) ( [sm_i qs_j C_ji] + sum_c p_c w_c^T + sum_{m<count} khat_m u_m^T ).
+ * The blob holds no pointers: copying it snapshots or restores a state (a
+ * prefix-cache entry after lq_window_flush is the prefix up to `pairs`).
+ * bits = 32 (the FP32-state reference): header, then f32 S[dk][dv] at 128.
+ */
+#ifndef LEAPQUANT_H
+#define LEAPQUANT_H
+
+#include <stddef.h>
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+#if defined(__GNUC__)
+#define LQ_API __attribute__((visibility("default")))
+#else
+#define LQ_API
+#endif
+
+/* Same object as cudaStream_t / CUstream; NULL is the legacy default stream. */
+typedef struct CUstream_st *lq_stream_t;
+
+typedef enum lq_status {
+    LQ_OK = 0,
+    LQ_ERR_INVALID_ARG = 1,  /* null pointer, non-positive size, bad enum     */
+    LQ_ERR_UNSUPPORTED = 2,  /* valid but not built: see lq_validate_config   */
+    LQ_ERR_CUDA = 3,         /* a CUDA call or launch failed                  */
+    LQ_ERR_WINDOW_FULL = 4,  /* device: decode step into a window of W pairs  */
+    LQ_ERR_RANGE = 5,        /* device: decay product left [2^-96, 1]         */
+    LQ_ERR_MISALIGNED = 6,   /* a pointer breaks the alignment rule above     */
+    LQ_ERR_TIMEOUT = 7,      /* device: an on-chip copy wait gave up          */
+    LQ_ERR_CORRUPT = 8       /* device: a blob header failed its checks       */
+} lq_status;
+
+/* Device status bits, ORed into a blob's status word. */
+#define LQ_DEV_WINDOW_FULL 0x1u
+#define LQ_DEV_RANGE 0x2u
+#define LQ_DEV_TIMEOUT 0x4u
+#define LQ_DEV_CORRUPT 0x8u
+
+typedef struct lq_config {
+    int32_t num_slots;   /* N > 0: independent sequences                      */
+    int32_t num_heads;   /* H > 0: heads per sequence (all of one kind)       */
+    int32_t dk, dv;      /* per-head state shape; built: dk == dv in {64,128} */
+    int32_t window;      /* W in [1, 64]: tokens per quantization window      */
+    int32_t num_comp;    /* r in [0, 16]: compensator lines                   */
+    int32_t bits;        /* 8, 6, 4 (LeapQuant state) or 32 (FP32 state)      */
+    int32_t decay_kind;  /* 0: GDN, one alpha per head; 1: KDA, a per key ch. */
+    int32_t scale_dtype; /* 0: qs/sm stored as f32; 1: as f16                 */
+    int32_t smoothing;   /* 1: per-key-row residual smoothing; 0: sm = 1      */
+    int32_t in_dtype;    /* q, k, v element type: 0 f32, 1 bf16               */
+} lq_config;
+
+/* LQ_OK if the configuration is valid and built, else why not.  Host only. */
+LQ_API lq_status lq_validate_config(const lq_config *cfg);
+
+/* Bytes of one (slot, head) blob, a multiple of 256; 0 for an invalid or
+ * unsupported configuration.  Host only. */
+LQ_API size_t lq_state_bytes(const lq_config *cfg);
+
+/* Enter a sequence: compress N*H dense FP32 states into the blobs.
+ *   state [N*H blobs]            out, overwritten entirely (header reset)
+ *   S0    [N, H, dk, dv] f32     in, row = key channel
+ * Runs the window-boundary compression (compensator extraction, smoothing,
+ * quantization) on S0; bits = 32 copies S0.  Source: the prefill state enters
+ * the quantized cache; per-window paragraph of the news post. */
+LQ_API lq_status lq_state_init(const lq_config *cfg, void *state, const float *S0, lq_stream_t stream);
+
+/* One decode token for every (slot, head).
+ *   state  [N*H blobs]           in/out: appends pair (khat_t, u_t), count++
+ *   q, k   [N, H, dk]  in_dtype  in
+ *   v      [N, H, dv]  in_dtype  in
+ *   beta   [N, H] f32            in, write strength
+ *   decay  [N, H] f32 (GDN: alpha) or [N, H, dk] f32 (KDA: a), in (0, 1]
+ *   out    [N, H, dv] f32        out, o_t = S_t^T q_t
+ * Outputs come from the fixed low-bit state, the compensators and the
+ * buffered pairs (abstract; per-window paragraph).  A (slot, head) whose
+ * window already holds W pairs, or whose status is nonzero, is skipped: its
+ * output row is written as zeros and its state is left unchanged.  Call
+ * lq_window_flush after every W steps. */
+LQ_API lq_status lq_decode_step(const lq_config *cfg, void *state, const void *q, const void *k,
+                         const void *v, const float *beta, const float *decay, float *out,
+                         lq_stream_t stream);
+
+/* Window boundary for every (slot, head): rebuild the FP32 state from the
+ * blob, extract r compensator lines, refresh the smoothing scales,
+ * requantize, and reset count = 0, g = 1 (news post: per-window, Compensator
+ * Tokens and residual smoothing paragraphs).  A (slot, head) with an empty
+ * window (count = 0) is left as is.  May be called on a partial window
+ * (sequence end, prefix-cache snapshot).  bits = 32: no-op. */
+LQ_API lq_status lq_window_flush(const lq_config *cfg, void *state, lq_stream_t stream);
+
+/* Write the dense FP32 state each blob stands for, pending pairs included:
+ *   S_out [N, H, dk, dv] f32, out.
+ * Evaluated exactly as the flush rebuilds it before requantizing, so the
+ * flush of a blob compresses bit-for-bit this matrix. */
+LQ_API lq_status lq_dequant_state(const lq_config *cfg, const void *state, float *S_out,
+                           lq_stream_t stream);
+
+/* Synchronize `stream`, OR the status words of all N*H blobs and map them to
+ * the first set error (WINDOW_FULL, RANGE, TIMEOUT, CORRUPT).  `state` is a
+ * device pointer; the read uses one strided device-to-host copy. */
+LQ_API lq_status lq_check_status(const lq_config *cfg, const void *state, lq_stream_t stream);
+
+/* Static text for a status code. */
+LQ_API const char *lq_status_string(lq_status s);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* LEAPQUANT_H */

@@ -1,0 +1,186 @@
+"""Python binding of libleapquant.so: argument marshalling only.
+
+Every function here has the name of the C entry point it calls (declared in
+include/leapquant.h), takes torch tensors (or raw integer addresses) and the
+current CUDA stream, and raises ``LQError`` on a non-zero status.  All
+arithmetic runs in the library's sm_100a kernels; there is no fallback path:
+if the library is missing, importing this module fails.
+"""
+from __future__ import annotations
+
+import ctypes
+import os
+
+_HERE = os.path.dirname(os.path.abspath(__file__))
+LIB_PATH = os.path.join(_HERE, "libleapquant.so")
+
+LQ_OK = 0
+STATUS_NAMES = {0: "LQ_OK", 1: "LQ_ERR_INVALID_ARG", 2: "LQ_ERR_UNSUPPORTED", 3: "LQ_ERR_CUDA",
+                4: "LQ_ERR_WINDOW_FULL", 5: "LQ_ERR_RANGE", 6: "LQ_ERR_MISALIGNED",
+                7: "LQ_ERR_TIMEOUT", 8: "LQ_ERR_CORRUPT"}
+ENTRY_POINTS = ("lq_validate_config", "lq_state_bytes", "lq_state_init", "lq_decode_step",
+                "lq_window_flush", "lq_dequant_state", "lq_check_status", "lq_status_string")
+
+
+class LQError(RuntimeError):
+    def __init__(self, status: int, where: str):
+        self.status = status
+        super().__init__(f"{where}: {STATUS_NAMES.get(status, status)} ({lq_status_string(status)})")
+
+
+class lq_config(ctypes.Structure):
+    _fields_ = [(n, ctypes.c_int32) for n in (
+        "num_slots", "num_heads", "dk", "dv", "window", "num_comp", "bits", "decay_kind",
+        "scale_dtype", "smoothing", "in_dtype")]
+
+    def __repr__(self):
+        return "lq_config(" + ", ".join(f"{n}={getattr(self, n)}" for n, _ in self._fields_) + ")"
+
+
+def make_config(num_slots, num_heads, dk=128, dv=128, window=16, num_comp=4, bits=8,
+                decay_kind="gdn", scale_dtype="f32", smoothing=True, in_dtype="bf16") -> lq_config:
+    return lq_config(int(num_slots), int(num_heads), int(dk), int(dv), int(window), int(num_comp),
+                     int(bits), 1 if decay_kind == "kda" else 0, 1 if scale_dtype == "f16" else 0,
+                     int(bool(smoothing)), 1 if in_dtype == "bf16" else 0)
+
+
+def config_for(wl, bits: int | None = None) -> lq_config:
+    """The lq_config of a generator Workload (optionally another bit width)."""
+    return make_config(wl.batch, wl.heads, wl.dk, wl.dv, wl.window, wl.num_comp,
+                       wl.bits if bits is None else bits, wl.decay_kind, wl.scale_dtype,
+                       wl.smoothing, wl.in_dtype)
+
+
+def _load():
+    if not os.path.exists(LIB_PATH):
+        raise ImportError(f"{LIB_PATH} is not built: run linear_attention_recurrent_lq_b200/build.py "
+                          "(or __graft_entry__.build())")
+    L = ctypes.CDLL(LIB_PATH)
+    P = ctypes.POINTER(lq_config)
+    vp, st = ctypes.c_void_p, ctypes.c_int
+    L.lq_validate_config.argtypes = [P]
+    L.lq_validate_config.restype = st
+    L.lq_state_bytes.argtypes = [P]
+    L.lq_state_bytes.restype = ctypes.c_size_t
+    L.lq_state_init.argtypes = [P, vp, vp, vp]
+    L.lq_state_init.restype = st
+    L.lq_decode_step.argtypes = [P, vp, vp, vp, vp, vp, vp, vp, vp]
+    L.lq_decode_step.restype = st
+    L.lq_window_flush.argtypes = [P, vp, vp]
+    L.lq_window_flush.restype = st
+    L.lq_dequant_state.argtypes = [P, vp, vp, vp]
+    L.lq_dequant_state.restype = st
+    L.lq_check_status.argtypes = [P, vp, vp]
+    L.lq_check_status.restype = st
+    L.lq_status_string.argtypes = [st]
+    L.lq_status_string.restype = ctypes.c_char_p
+    return L
+
+
+lib = _load()
+
+
+def _ptr(x) -> int | None:
+    if x is None:
+        return None
+    if isinstance(x, int):
+        return x
+    if not x.is_contiguous():
+        raise ValueError("tensors passed to the library must be contiguous")
+    return x.data_ptr()
+
+
+def _stream(stream) -> int | None:
+    if stream is None:
+        import torch
+        if not torch.cuda.is_available():
+            return None
+        return torch.cuda.current_stream().cuda_stream
+    if isinstance(stream, int):
+        return stream
+    return stream.cuda_stream
+
+
+def _check(status: int, where: str):
+    if status != LQ_OK:
+        raise LQError(status, where)
+
+
+def lq_status_string(status: int) -> str:
+    return lib.lq_status_string(int(status)).decode()
+
+
+def lq_validate_config(cfg: lq_config) -> int:
+    return lib.lq_validate_config(ctypes.byref(cfg))
+
+
+def lq_state_bytes(cfg: lq_config) -> int:
+    n = lib.lq_state_bytes(ctypes.byref(cfg))
+    if n == 0:
+        _check(lq_validate_config(cfg) or 1, "lq_state_bytes")
+    return n
+
+
+def lq_state_init(cfg, state, S0, stream=None):
+    _check(lib.lq_state_init(ctypes.byref(cfg), _ptr(state), _ptr(S0), _stream(stream)),
+           "lq_state_init")
+
+
+def lq_decode_step(cfg, state, q, k, v, beta, decay, out, stream=None):
+    _check(lib.lq_decode_step(ctypes.byref(cfg), _ptr(state), _ptr(q), _ptr(k), _ptr(v),
+                              _ptr(beta), _ptr(decay), _ptr(out), _stream(stream)),
+           "lq_decode_step")
+
+
+def lq_window_flush(cfg, state, stream=None):
+    _check(lib.lq_window_flush(ctypes.byref(cfg), _ptr(state), _stream(stream)), "lq_window_flush")
+
+
+def lq_dequant_state(cfg, state, S_out, stream=None):
+    _check(lib.lq_dequant_state(ctypes.byref(cfg), _ptr(state), _ptr(S_out), _stream(stream)),
+           "lq_dequant_state")
+
+
+def lq_check_status(cfg, state, stream=None) -> int:
+    """Synchronizes the stream; returns the status code (does not raise)."""
+    return lib.lq_check_status(ctypes.byref(cfg), _ptr(state), _stream(stream))
+
+
+class LQState:
+    """N*H state blobs in one device buffer, with the library's calls bound."""
+
+    def __init__(self, cfg: lq_config, device="cuda"):
+        import torch
+        self.cfg = cfg
+        self.blob_bytes = lq_state_bytes(cfg)
+        self.buf = torch.empty(cfg.num_slots * cfg.num_heads * self.blob_bytes, dtype=torch.uint8,
+                               device=device)
+
+    @property
+    def ptr(self) -> int:
+        return self.buf.data_ptr()
+
+    def blobs(self):
+        """[N*H, blob_bytes] uint8 view."""
+        return self.buf.view(-1, self.blob_bytes)
+
+    def init(self, S0, stream=None):
+        lq_state_init(self.cfg, self.buf, S0, stream)
+
+    def step(self, q, k, v, beta, decay, out, stream=None):
+        lq_decode_step(self.cfg, self.buf, q, k, v, beta, decay, out, stream)
+
+    def flush(self, stream=None):
+        lq_window_flush(self.cfg, self.buf, stream)
+
+    def dequant(self, S_out=None, stream=None):
+        import torch
+        c = self.cfg
+        if S_out is None:
+            S_out = torch.empty((c.num_slots, c.num_heads, c.dk, c.dv), dtype=torch.float32,
+                                device=self.buf.device)
+        lq_dequant_state(c, self.buf, S_out, stream)
+        return S_out
+
+    def check(self, stream=None) -> int:
+        return lq_check_status(self.cfg, self.buf, stream)

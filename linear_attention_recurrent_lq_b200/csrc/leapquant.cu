@@ -1,0 +1,242 @@
+// leapquant.cu -- host side of the C ABI declared in include/leapquant.h:
+// argument checks, blob layout, and launches of the sm_100a kernels.
+#include <cuda_runtime.h>
+#include <stdint.h>
+
+#include <mutex>
+#include <vector>
+
+#include "leapquant.h"
+#include "lq_common.cuh"
+#include "lq_decode.cuh"
+#include "lq_flush.cuh"
+#include "lq_fp32.cuh"
+
+using namespace lq;
+
+namespace {
+
+bool aligned(const void *p, uintptr_t a) { return (reinterpret_cast<uintptr_t>(p) % a) == 0; }
+
+lq_status check_config(const lq_config *c) {
+    if (!c) return LQ_ERR_INVALID_ARG;
+    if (c->num_slots <= 0 || c->num_heads <= 0 || c->dk <= 0 || c->dv <= 0 || c->window <= 0 ||
+        c->num_comp < 0)
+        return LQ_ERR_INVALID_ARG;
+    if (c->bits != 4 && c->bits != 6 && c->bits != 8 && c->bits != 32) return LQ_ERR_INVALID_ARG;
+    if ((c->decay_kind | c->scale_dtype | c->smoothing | c->in_dtype) & ~1) return LQ_ERR_INVALID_ARG;
+    if ((int64_t)c->num_slots * c->num_heads > 0x7FFFFFFF) return LQ_ERR_UNSUPPORTED;
+    if (c->dk != c->dv || (c->dk != 64 && c->dk != 128)) return LQ_ERR_UNSUPPORTED;
+    if (c->window > kMaxWindow || c->num_comp > kMaxComp) return LQ_ERR_UNSUPPORTED;
+    return LQ_OK;
+}
+
+Flags make_flags(const lq_config &c) {
+    return Flags{c.decay_kind, c.scale_dtype, c.in_dtype, c.smoothing, c.window, c.num_comp};
+}
+
+// Allow a kernel more than 48 KB of dynamic shared memory, once per device.
+template <typename K>
+cudaError_t allow_smem(K kernel, uint32_t bytes) {
+    static std::mutex mu;
+    static std::vector<std::pair<int, uint32_t>> done;  // (device, bytes already allowed)
+    if (bytes <= 48u * 1024u) return cudaSuccess;
+    int dev = 0;
+    cudaError_t e = cudaGetDevice(&dev);
+    if (e != cudaSuccess) return e;
+    std::lock_guard<std::mutex> lock(mu);
+    for (auto &d : done)
+        if (d.first == dev && d.second >= bytes) return cudaSuccess;
+    e = cudaFuncSetAttribute(kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)bytes);
+    if (e == cudaSuccess) done.push_back({dev, bytes});
+    return e;
+}
+
+lq_status launched(cudaError_t e) {
+    if (e != cudaSuccess) return LQ_ERR_CUDA;
+    return cudaGetLastError() == cudaSuccess ? LQ_OK : LQ_ERR_CUDA;
+}
+
+template <int D, int BITS>
+lq_status launch_decode(const lq_config &c, const DecodeArgs &a, cudaStream_t s) {
+    const uint32_t smem = decode_smem_bytes(D, a.L, c.window);
+    auto k = decode_kernel<D, BITS>;
+    cudaError_t e = allow_smem(k, smem);
+    if (e != cudaSuccess) return LQ_ERR_CUDA;
+    k<<<(unsigned)(c.num_slots * c.num_heads), 2 * D, smem, s>>>(a);
+    return launched(cudaSuccess);
+}
+
+template <int D, int BITS, int MODE>
+lq_status launch_boundary(const lq_config &c, const FlushArgs &a, cudaStream_t s) {
+    const uint32_t smem = flush_smem_bytes(D, BITS, a.L, c.window, c.decay_kind);
+    auto k = boundary_kernel<D, BITS, MODE>;
+    cudaError_t e = allow_smem(k, smem);
+    if (e != cudaSuccess) return LQ_ERR_CUDA;
+    k<<<(unsigned)(c.num_slots * c.num_heads), 4 * D, smem, s>>>(a);
+    return launched(cudaSuccess);
+}
+
+template <int MODE>
+lq_status dispatch_boundary(const lq_config &c, const FlushArgs &a, cudaStream_t s) {
+    switch (c.dk * 100 + c.bits) {
+        case 12808: return launch_boundary<128, 8, MODE>(c, a, s);
+        case 12806: return launch_boundary<128, 6, MODE>(c, a, s);
+        case 12804: return launch_boundary<128, 4, MODE>(c, a, s);
+        case 6408: return launch_boundary<64, 8, MODE>(c, a, s);
+        case 6406: return launch_boundary<64, 6, MODE>(c, a, s);
+        case 6404: return launch_boundary<64, 4, MODE>(c, a, s);
+        default: return LQ_ERR_UNSUPPORTED;
+    }
+}
+
+template <int D>
+lq_status launch_fp32_decode(const lq_config &c, const Fp32Args &a, cudaStream_t s) {
+    const uint32_t smem = fp32_smem_bytes<D>();
+    auto k = fp32_decode_kernel<D>;
+    cudaError_t e = allow_smem(k, smem);
+    if (e != cudaSuccess) return LQ_ERR_CUDA;
+    k<<<(unsigned)(c.num_slots * c.num_heads), 4 * D, smem, s>>>(a);
+    return launched(cudaSuccess);
+}
+
+template <int MODE>
+lq_status launch_fp32_copy(const lq_config &c, const Fp32Args &a, cudaStream_t s) {
+    const unsigned grid = (unsigned)(c.num_slots * c.num_heads);
+    if (c.dk == 128)
+        fp32_copy_kernel<128, MODE><<<grid, 256, 0, s>>>(a);
+    else
+        fp32_copy_kernel<64, MODE><<<grid, 256, 0, s>>>(a);
+    return launched(cudaSuccess);
+}
+
+}  // namespace
+
+extern "C" {
+
+lq_status lq_validate_config(const lq_config *cfg) { return check_config(cfg); }
+
+size_t lq_state_bytes(const lq_config *cfg) {
+    if (check_config(cfg) != LQ_OK) return 0;
+    return make_layout(*cfg).blob;
+}
+
+lq_status lq_state_init(const lq_config *cfg, void *state, const float *S0, lq_stream_t stream) {
+    lq_status st = check_config(cfg);
+    if (st != LQ_OK) return st;
+    if (!state || !S0) return LQ_ERR_INVALID_ARG;
+    if (!aligned(state, 256) || !aligned(S0, 16)) return LQ_ERR_MISALIGNED;
+    const lq_config &c = *cfg;
+    const Layout L = make_layout(c);
+    cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
+    if (c.bits == 32) {
+        Fp32Args a{};
+        a.state = static_cast<uint8_t *>(state);
+        a.S0 = S0;
+        a.L = L;
+        return launch_fp32_copy<1>(c, a, s);
+    }
+    FlushArgs a{static_cast<uint8_t *>(state), S0, nullptr, L, make_flags(c)};
+    return dispatch_boundary<1>(c, a, s);
+}
+
+lq_status lq_decode_step(const lq_config *cfg, void *state, const void *q, const void *k,
+                         const void *v, const float *beta, const float *decay, float *out,
+                         lq_stream_t stream) {
+    lq_status st = check_config(cfg);
+    if (st != LQ_OK) return st;
+    if (!state || !q || !k || !v || !beta || !decay || !out) return LQ_ERR_INVALID_ARG;
+    if (!aligned(state, 256) || !aligned(q, 16) || !aligned(k, 16) || !aligned(v, 16) ||
+        !aligned(beta, 16) || !aligned(decay, 16) || !aligned(out, 16))
+        return LQ_ERR_MISALIGNED;
+    const lq_config &c = *cfg;
+    const Layout L = make_layout(c);
+    cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
+    if (c.bits == 32) {
+        Fp32Args a{static_cast<uint8_t *>(state), nullptr, nullptr, L, make_flags(c), q, k, v,
+                   beta, decay, out};
+        return c.dk == 128 ? launch_fp32_decode<128>(c, a, s) : launch_fp32_decode<64>(c, a, s);
+    }
+    DecodeArgs a{static_cast<uint8_t *>(state), L, make_flags(c), q, k, v, beta, decay, out};
+    switch (c.dk * 100 + c.bits) {
+        case 12808: return launch_decode<128, 8>(c, a, s);
+        case 12806: return launch_decode<128, 6>(c, a, s);
+        case 12804: return launch_decode<128, 4>(c, a, s);
+        case 6408: return launch_decode<64, 8>(c, a, s);
+        case 6406: return launch_decode<64, 6>(c, a, s);
+        case 6404: return launch_decode<64, 4>(c, a, s);
+        default: return LQ_ERR_UNSUPPORTED;
+    }
+}
+
+lq_status lq_window_flush(const lq_config *cfg, void *state, lq_stream_t stream) {
+    lq_status st = check_config(cfg);
+    if (st != LQ_OK) return st;
+    if (!state) return LQ_ERR_INVALID_ARG;
+    if (!aligned(state, 256)) return LQ_ERR_MISALIGNED;
+    const lq_config &c = *cfg;
+    if (c.bits == 32) return LQ_OK;
+    FlushArgs a{static_cast<uint8_t *>(state), nullptr, nullptr, make_layout(c), make_flags(c)};
+    return dispatch_boundary<0>(c, a, reinterpret_cast<cudaStream_t>(stream));
+}
+
+lq_status lq_dequant_state(const lq_config *cfg, const void *state, float *S_out, lq_stream_t stream) {
+    lq_status st = check_config(cfg);
+    if (st != LQ_OK) return st;
+    if (!state || !S_out) return LQ_ERR_INVALID_ARG;
+    if (!aligned(state, 256) || !aligned(S_out, 16)) return LQ_ERR_MISALIGNED;
+    const lq_config &c = *cfg;
+    const Layout L = make_layout(c);
+    cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
+    uint8_t *st8 = const_cast<uint8_t *>(static_cast<const uint8_t *>(state));
+    if (c.bits == 32) {
+        Fp32Args a{};
+        a.state = st8;
+        a.S_out = S_out;
+        a.L = L;
+        return launch_fp32_copy<2>(c, a, s);
+    }
+    FlushArgs a{st8, nullptr, S_out, L, make_flags(c)};
+    return dispatch_boundary<2>(c, a, s);
+}
+
+lq_status lq_check_status(const lq_config *cfg, const void *state, lq_stream_t stream) {
+    lq_status st = check_config(cfg);
+    if (st != LQ_OK) return st;
+    if (!state) return LQ_ERR_INVALID_ARG;
+    if (!aligned(state, 256)) return LQ_ERR_MISALIGNED;
+    const lq_config &c = *cfg;
+    const Layout L = make_layout(c);
+    const size_t n = (size_t)c.num_slots * c.num_heads;
+    std::vector<uint32_t> words(n);
+    cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
+    cudaError_t e = cudaMemcpy2DAsync(words.data(), sizeof(uint32_t),
+                                      static_cast<const uint8_t *>(state) + kHdrStatus, L.blob,
+                                      sizeof(uint32_t), n, cudaMemcpyDeviceToHost, s);
+    if (e == cudaSuccess) e = cudaStreamSynchronize(s);
+    if (e != cudaSuccess) return LQ_ERR_CUDA;
+    uint32_t any = 0;
+    for (uint32_t w : words) any |= w;
+    if (any & LQ_DEV_WINDOW_FULL) return LQ_ERR_WINDOW_FULL;
+    if (any & LQ_DEV_RANGE) return LQ_ERR_RANGE;
+    if (any & LQ_DEV_TIMEOUT) return LQ_ERR_TIMEOUT;
+    if (any & LQ_DEV_CORRUPT) return LQ_ERR_CORRUPT;
+    return LQ_OK;
+}
+
+const char *lq_status_string(lq_status s) {
+    switch (s) {
+        case LQ_OK: return "ok";
+        case LQ_ERR_INVALID_ARG: return "invalid argument";
+        case LQ_ERR_UNSUPPORTED: return "configuration not supported by this build";
+        case LQ_ERR_CUDA: return "CUDA error";
+        case LQ_ERR_WINDOW_FULL: return "decode step into a full window (flush every W steps)";
+        case LQ_ERR_RANGE: return "window decay product fell below 2^-96";
+        case LQ_ERR_MISALIGNED: return "pointer misaligned (state: 256 B, others: 16 B)";
+        case LQ_ERR_TIMEOUT: return "on-chip copy wait timed out";
+        case LQ_ERR_CORRUPT: return "state blob header failed its checks";
+    }
+    return "unknown status";
+}
+
+}  // extern "C"

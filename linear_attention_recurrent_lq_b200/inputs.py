@@ -217,3 +217,19 @@ def draw(wl: Workload, n_tokens: int | None = None, stream: int = 0) -> dict:
     st = s.state()
     st.update(s.tokens(wl.tokens if n_tokens is None else n_tokens))
     return st
+
+
+def to_device(wl: Workload, d: dict, device="cuda") -> dict:
+    """Upload drawn tokens as the tensors the library reads: q, k, v in the
+    workload's input dtype (bf16 as its bit patterns), beta and decay f32."""
+    import torch
+    dev = {}
+    for name in ("q", "k", "v"):
+        if wl.in_dtype == "bf16":
+            bits = np.ascontiguousarray(d[name + "_bits"]).view(np.int16)
+            dev[name] = torch.from_numpy(bits).to(device).view(torch.bfloat16)
+        else:
+            dev[name] = torch.from_numpy(np.ascontiguousarray(d[name])).to(device)
+    dev["beta"] = torch.from_numpy(np.ascontiguousarray(d["beta"])).to(device)
+    dev["decay"] = torch.from_numpy(np.ascontiguousarray(d["decay"])).to(device)
+    return dev

@@ -1,0 +1,87 @@
+"""Host-side checks of the C ABI that need no GPU: the library loads, exports
+every entry point include/leapquant.h declares, sizes blobs as documented,
+and rejects bad arguments before launching anything."""
+import ctypes
+import os
+import re
+
+import pytest
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+HEADER = os.path.join(ROOT, "include", "leapquant.h")
+
+
+@pytest.fixture(scope="module")
+def B():
+    from linear_attention_recurrent_lq_b200 import build
+    build.build()
+    from linear_attention_recurrent_lq_b200 import binding
+    return binding
+
+
+def declared_functions():
+    text = open(HEADER).read()
+    return re.findall(r"^LQ_API\s+[\w\s\*]+?\b(lq_\w+)\s*\(", text, flags=re.M)
+
+
+def test_library_exports_every_declared_entry_point(B):
+    names = declared_functions()
+    assert set(names) == set(B.ENTRY_POINTS)
+    lib = ctypes.CDLL(B.LIB_PATH)
+    for n in names:
+        assert hasattr(lib, n), n
+
+
+def test_state_bytes_follow_documented_layout(B):
+    from tests import blob
+    for bits in (8, 6, 4):
+        for kda in (0, 1):
+            for f16 in (0, 1):
+                for d in (64, 128):
+                    for w, r in ((16, 4), (1, 0), (64, 16)):
+                        cfg = B.make_config(2, 3, d, d, w, r, bits, "kda" if kda else "gdn",
+                                            "f16" if f16 else "f32")
+                        L = blob.layout(d, d, w, r, bits, kda, f16)
+                        assert B.lq_state_bytes(cfg) == L.blob
+                        assert L.blob % 256 == 0
+    cfg = B.make_config(64, 32, bits=32)
+    assert B.lq_state_bytes(cfg) == blob.layout(128, 128, 16, 4, 32, 0, 0).blob
+
+
+def test_headline_blob_size(B):
+    # GDN, INT8, dk = dv = 128, W = 16, r = 4, f32 scales
+    assert B.lq_state_bytes(B.make_config(64, 32)) == 36096
+
+
+@pytest.mark.parametrize("field,value,expect", [
+    ("num_slots", 0, 1), ("num_heads", -1, 1), ("window", 0, 1), ("bits", 5, 1),
+    ("decay_kind", 2, 1), ("scale_dtype", 3, 1), ("num_comp", -1, 1),
+    ("dk", 256, 2), ("dv", 64, 2), ("window", 65, 2), ("num_comp", 17, 2)])
+def test_config_validation(B, field, value, expect):
+    cfg = B.make_config(4, 4)
+    setattr(cfg, field, value)
+    assert B.lq_validate_config(cfg) == expect
+    assert B.lib.lq_state_bytes(ctypes.byref(cfg)) == 0
+
+
+def test_null_and_misaligned_pointers_rejected_before_launch(B):
+    cfg = B.make_config(4, 4)
+    L = B.lib
+    c = ctypes.byref(cfg)
+    assert L.lq_decode_step(c, None, 16, 16, 16, 16, 16, 16, None) == 1
+    assert L.lq_decode_step(c, 256, 16, 16, 16, 16, 16, None, None) == 1
+    assert L.lq_decode_step(c, 128, 16, 16, 16, 16, 16, 16, None) == 6   # state needs 256 B
+    assert L.lq_decode_step(c, 256, 8, 16, 16, 16, 16, 16, None) == 6    # q needs 16 B
+    assert L.lq_state_init(c, 256, 4, None) == 6
+    assert L.lq_state_init(c, None, 16, None) == 1
+    assert L.lq_window_flush(c, 100, None) == 6
+    assert L.lq_window_flush(c, None, None) == 1
+    assert L.lq_dequant_state(c, 256, 12, None) == 6
+    assert L.lq_check_status(c, None, None) == 1
+    assert L.lq_decode_step(None, 256, 16, 16, 16, 16, 16, 16, None) == 1
+
+
+def test_status_strings(B):
+    for code in range(9):
+        assert B.lq_status_string(code)
+    assert B.lq_status_string(99) == "unknown status"
