@@ -32,9 +32,10 @@
  *    then skip that (slot, head) and never trap.  lq_check_status reads them.
  *  - Tensors are dense, row-major, contiguous.  N = num_slots (sequences),
  *    H = num_heads.  The state buffer holds N*H consecutive blobs of
- *    lq_state_bytes(cfg) bytes each, blob (n, h) at index n*H + h.  Pointers
- *    must be 16-byte aligned and the state buffer 256-byte aligned
- *    (LQ_ERR_MISALIGNED otherwise).
+ *    lq_state_bytes(cfg) bytes each, blob (n, h) at index n*H + h.
+ *    Alignment (LQ_ERR_MISALIGNED otherwise): the state buffer 256 bytes;
+ *    q, k, v, S0, S_out and a KDA decay 16 bytes; beta, a GDN decay and out
+ *    4 bytes.
  *  - Calls on one state must be ordered (same stream or explicit events);
  *    calls on disjoint states may run concurrently.
  *

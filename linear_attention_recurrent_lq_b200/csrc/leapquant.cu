@@ -35,20 +35,28 @@ Flags make_flags(const lq_config &c) {
     return Flags{c.decay_kind, c.scale_dtype, c.in_dtype, c.smoothing, c.window, c.num_comp};
 }
 
-// Allow a kernel more than 48 KB of dynamic shared memory, once per device.
+// Allow a kernel more than 48 KB of dynamic shared memory (once per kernel
+// and device).
+struct SmemGrant {
+    int dev;
+    const void *fn;
+    uint32_t bytes;
+};
+
 template <typename K>
 cudaError_t allow_smem(K kernel, uint32_t bytes) {
     static std::mutex mu;
-    static std::vector<std::pair<int, uint32_t>> done;  // (device, bytes already allowed)
+    static std::vector<SmemGrant> done;
     if (bytes <= 48u * 1024u) return cudaSuccess;
     int dev = 0;
     cudaError_t e = cudaGetDevice(&dev);
     if (e != cudaSuccess) return e;
+    const void *fn = reinterpret_cast<const void *>(kernel);
     std::lock_guard<std::mutex> lock(mu);
-    for (auto &d : done)
-        if (d.first == dev && d.second >= bytes) return cudaSuccess;
+    for (const SmemGrant &g : done)
+        if (g.dev == dev && g.fn == fn && g.bytes >= bytes) return cudaSuccess;
     e = cudaFuncSetAttribute(kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)bytes);
-    if (e == cudaSuccess) done.push_back({dev, bytes});
+    if (e == cudaSuccess) done.push_back({dev, fn, bytes});
     return e;
 }
 
@@ -147,7 +155,7 @@ lq_status lq_decode_step(const lq_config *cfg, void *state, const void *q, const
     if (st != LQ_OK) return st;
     if (!state || !q || !k || !v || !beta || !decay || !out) return LQ_ERR_INVALID_ARG;
     if (!aligned(state, 256) || !aligned(q, 16) || !aligned(k, 16) || !aligned(v, 16) ||
-        !aligned(beta, 16) || !aligned(decay, 16) || !aligned(out, 16))
+        !aligned(beta, 4) || !aligned(decay, cfg->decay_kind ? 16 : 4) || !aligned(out, 4))
         return LQ_ERR_MISALIGNED;
     const lq_config &c = *cfg;
     const Layout L = make_layout(c);
@@ -232,7 +240,7 @@ const char *lq_status_string(lq_status s) {
         case LQ_ERR_CUDA: return "CUDA error";
         case LQ_ERR_WINDOW_FULL: return "decode step into a full window (flush every W steps)";
         case LQ_ERR_RANGE: return "window decay product fell below 2^-96";
-        case LQ_ERR_MISALIGNED: return "pointer misaligned (state: 256 B, others: 16 B)";
+        case LQ_ERR_MISALIGNED: return "pointer misaligned (see the alignment rule in leapquant.h)";
         case LQ_ERR_TIMEOUT: return "on-chip copy wait timed out";
         case LQ_ERR_CORRUPT: return "state blob header failed its checks";
     }

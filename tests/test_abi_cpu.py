@@ -72,6 +72,7 @@ def test_null_and_misaligned_pointers_rejected_before_launch(B):
     assert L.lq_decode_step(c, 256, 16, 16, 16, 16, 16, None, None) == 1
     assert L.lq_decode_step(c, 128, 16, 16, 16, 16, 16, 16, None) == 6   # state needs 256 B
     assert L.lq_decode_step(c, 256, 8, 16, 16, 16, 16, 16, None) == 6    # q needs 16 B
+    assert L.lq_decode_step(c, 256, 16, 16, 16, 2, 16, 16, None) == 6    # beta needs 4 B
     assert L.lq_state_init(c, 256, 4, None) == 6
     assert L.lq_state_init(c, None, 16, None) == 1
     assert L.lq_window_flush(c, 100, None) == 6
