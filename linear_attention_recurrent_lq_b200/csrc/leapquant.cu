@@ -65,13 +65,43 @@ lq_status launched(cudaError_t e) {
     return cudaGetLastError() == cudaSuccess ? LQ_OK : LQ_ERR_CUDA;
 }
 
+// Persistent grid: as many CTAs as fit on the device at once, each walking
+// a strided list of (slot, head) blobs.
+template <typename K>
+int persistent_grid(K kernel, int threads, uint32_t smem, int work) {
+    static std::mutex mu;
+    static std::vector<std::pair<std::pair<const void *, uint32_t>, int>> cache;
+    const void *fn = reinterpret_cast<const void *>(kernel);
+    int per_sm = 0, sms = 0, dev = 0;
+    {
+        std::lock_guard<std::mutex> lock(mu);
+        for (auto &e : cache)
+            if (e.first.first == fn && e.first.second == smem) per_sm = e.second;
+    }
+    if (cudaGetDevice(&dev) != cudaSuccess ||
+        cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess)
+        return -1;
+    if (per_sm == 0) {
+        if (cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, kernel, threads, smem) != cudaSuccess)
+            return -1;
+        if (per_sm < 1) per_sm = 1;
+        std::lock_guard<std::mutex> lock(mu);
+        cache.push_back({{fn, smem}, per_sm});
+    }
+    const long cap = (long)sms * per_sm;
+    return (int)(work < cap ? work : cap);
+}
+
 template <int D, int BITS>
 lq_status launch_decode(const lq_config &c, const DecodeArgs &a, cudaStream_t s) {
-    const uint32_t smem = decode_smem_bytes(D, a.L, c.window);
+    const uint32_t smem = decode_smem_bytes(D, a.L, a.F);
     auto k = decode_kernel<D, BITS>;
     cudaError_t e = allow_smem(k, smem);
     if (e != cudaSuccess) return LQ_ERR_CUDA;
-    k<<<(unsigned)(c.num_slots * c.num_heads), 2 * D, smem, s>>>(a);
+    const int threads = D + 32;
+    const int grid = persistent_grid(k, threads, smem, a.num_heads);
+    if (grid <= 0) return LQ_ERR_CUDA;
+    k<<<grid, threads, smem, s>>>(a);
     return launched(cudaSuccess);
 }
 
@@ -165,7 +195,8 @@ lq_status lq_decode_step(const lq_config *cfg, void *state, const void *q, const
                    beta, decay, out};
         return c.dk == 128 ? launch_fp32_decode<128>(c, a, s) : launch_fp32_decode<64>(c, a, s);
     }
-    DecodeArgs a{static_cast<uint8_t *>(state), L, make_flags(c), q, k, v, beta, decay, out};
+    DecodeArgs a{static_cast<uint8_t *>(state), L, make_flags(c), q, k, v, beta, decay, out,
+                 c.num_slots * c.num_heads};
     switch (c.dk * 100 + c.bits) {
         case 12808: return launch_decode<128, 8>(c, a, s);
         case 12806: return launch_decode<128, 6>(c, a, s);

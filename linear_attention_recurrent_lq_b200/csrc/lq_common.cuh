@@ -100,25 +100,32 @@ __device__ __forceinline__ void mbar_arrive_expect_tx(uint64_t *bar, uint32_t by
                  "r"(bytes) : "memory");
 }
 
+// Test for completion of phase `phase`; the thread may sleep in the barrier
+// for up to ~1 ms (suspend-time hint) while the phase is still open.
 __device__ __forceinline__ bool mbar_try_wait(uint64_t *bar, uint32_t phase) {
     uint32_t ok;
     asm volatile(
         "{\n\t.reg .pred p;\n\t"
-        "mbarrier.try_wait.parity.shared::cta.b64 p, [%1], %2;\n\t"
+        "mbarrier.try_wait.parity.shared::cta.b64 p, [%1], %2, %3;\n\t"
         "selp.u32 %0, 1, 0, p;\n\t}"
         : "=r"(ok)
-        : "r"(smem_u32(bar)), "r"(phase)
+        : "r"(smem_u32(bar)), "r"(phase), "r"(1000000u)
         : "memory");
     return ok != 0;
+}
+
+__device__ __forceinline__ void mbar_arrive(uint64_t *bar) {
+    asm volatile("mbarrier.arrive.shared::cta.b64 _, [%0];" ::"r"(smem_u32(bar)) : "memory");
 }
 
 // Wait for phase `phase` of `bar`, giving up after kWaitLimitNs.  Returns
 // false on timeout (the caller records it and returns; it never spins on).
 __device__ __noinline__ bool mbar_wait_bounded(uint64_t *bar, uint32_t phase) {
+    if (mbar_try_wait(bar, phase)) return true;
     const unsigned long long t0 = global_ns();
-    for (uint32_t it = 0;; ++it) {
+    for (;;) {
         if (mbar_try_wait(bar, phase)) return true;
-        if ((it & 7u) == 7u && global_ns() - t0 > kWaitLimitNs) return false;
+        if (global_ns() - t0 > kWaitLimitNs) return false;
     }
 }
 

@@ -15,13 +15,24 @@
 //     u_t = beta (v - a),   o_t = b + (k . q) u_t,
 // and the pair (khat_t = k / g_t, u_t) is appended.
 //
-// One CTA per (slot, head), 2*D threads.  Thread 0 starts two bulk copies
-// into shared memory (scales + compensators + codes at once, then the buffered
-// pairs once the header says how many), while all threads load q, k, v and
-// build the decay-folded vectors.  The GEMV reads 16-code groups from shared
-// memory (conflict-free for 8, 6 and 4 bits), turns codes into exact floats
-// with byte permutes instead of int->float conversions, and reduces over the
-// D/16 threads of a row with a reduce-scatter shuffle tree.
+// Persistent kernel, one CTA = D consumer threads + one producer warp, each
+// CTA walking a strided list of (slot, head) blobs:
+//  * the producer warp bulk-copies each blob's small, variable-size parts
+//    (header, decay product, scales, compensators, the buffered pairs) and the
+//    token's q, k, v into a two-stage shared-memory ring (mbarrier-tracked);
+//  * the codes (the bulk of the state) go straight from global memory into
+//    registers: a consumer thread holds its D/16 16-code groups of the current
+//    blob and, as it consumes group m, issues the load of group m of the next
+//    blob, so code traffic is always in flight;
+//  * the GEMV runs on the integer pipe: x_k, x_q are quantized per 16-key
+//    chunk to int16 with the chunk's own scale (error <= 2^-16 of the chunk's
+//    largest entry) and dp2a multiplies two int16 entries by two int8 codes,
+//    accumulating exactly in int32;
+//  * a row is split over D/16 threads (one chunk each); a reduce-scatter over
+//    them leaves each thread with (a_j, b_j) of one row j, to which it adds
+//    the compensator and pair terms from shared memory before forming u_j and
+//    o_j.  Waits on the ring sleep on the mbarrier and give up after a bounded
+//    time.
 #pragma once
 
 #include "lq_common.cuh"
@@ -35,34 +46,185 @@ struct DecodeArgs {
     const void *q, *k, *v;
     const float *beta, *decay;
     float *out;
+    int num_heads;  // N * H
 };
 
 constexpr int kDotSlots = kMaxWindow + kMaxComp;
 
+// One ring stage: [blob prefix up to the codes][buffered pairs][q k v][KDA decay][aux]
+struct DecodeStage {
+    uint32_t pairs_at, in_off, qkv_bytes, dec_off, aux_off, bytes;
+};
+
+__host__ __device__ inline DecodeStage decode_stage(const Layout &L, int D, int window, int bf16,
+                                                    int kda) {
+    DecodeStage S;
+    S.pairs_at = L.codes_off;  // the prefix [0, codes_off) is copied as is
+    S.in_off = align_up(S.pairs_at + (uint32_t)(window - 1) * L.pair_bytes, 128);
+    S.qkv_bytes = align_up((uint32_t)D * (bf16 ? 2u : 4u), 16);
+    S.dec_off = S.in_off + 3 * S.qkv_bytes;
+    S.aux_off = align_up(S.dec_off + (kda ? (uint32_t)D * 4u : 0u), 16);
+    S.bytes = align_up(S.aux_off + 16, 128);
+    return S;
+}
+
 template <int D>
 __host__ __device__ constexpr uint32_t decode_fixed_smem() {
-    // barriers + header (128), y/x/gemv (6D floats), dots (2*kDotSlots), reduce (32)
-    return align_up(128u + (6u * D + 2u * kDotSlots + 32u) * 4u, 128u);
+    // barriers + control (128) | y [2D] | X int16 [2D] | chunk scales [2*D/16] | dots [2*kDotSlots]
+    // | column terms [2D] | new keys [D] | new decay [D] | reduce [32] | producer batch [3*32]
+    // | comp lists [2*16] | info [8]
+    return align_up(128u + (2u * D + D + 2u * (D / 16) + 2u * kDotSlots + 2u * D + 2u * D + 32u +
+                            96u + 32u + 8u) * 4u, 128u);
 }
 
-inline uint32_t decode_smem_bytes(int D, const Layout &L, int window) {
+constexpr int kDecodeStages = 2;
+
+inline uint32_t decode_smem_bytes(int D, const Layout &L, const Flags &F) {
     const uint32_t fixed = D == 128 ? decode_fixed_smem<128>() : decode_fixed_smem<64>();
-    return fixed + align_up(L.compact_bytes, 128) + (uint32_t)(window - 1) * L.pair_bytes;
+    return fixed + (uint32_t)kDecodeStages * decode_stage(L, D, F.window, F.bf16_in, F.kda).bytes;
 }
 
-// Reduce-scatter of N values over the N consecutive lanes of an aligned
+__device__ __forceinline__ void consumer_sync(int n) {
+    asm volatile("bar.sync 1, %0;" ::"r"(n) : "memory");
+}
+
+__device__ __forceinline__ bool consumer_sync_or(bool pred, int n) {
+    uint32_t r;
+    asm volatile(
+        "{\n\t.reg .pred p, q;\n\t"
+        "setp.ne.u32 p, %1, 0;\n\t"
+        "bar.red.or.pred q, 1, %2, p;\n\t"
+        "selp.u32 %0, 1, 0, q;\n\t}"
+        : "=r"(r)
+        : "r"((uint32_t)pred), "r"(n)
+        : "memory");
+    return r != 0;
+}
+
+__device__ __forceinline__ bool consumer_sync_and(bool pred, int n) {
+    uint32_t r;
+    asm volatile(
+        "{\n\t.reg .pred p, q;\n\t"
+        "setp.ne.u32 p, %1, 0;\n\t"
+        "bar.red.and.pred q, 1, %2, p;\n\t"
+        "selp.u32 %0, 1, 0, q;\n\t}"
+        : "=r"(r)
+        : "r"((uint32_t)pred), "r"(n)
+        : "memory");
+    return r != 0;
+}
+
+__device__ __forceinline__ int dp2a_lo_ss(uint32_t a, uint32_t b, int c) {
+    int d;
+    asm("dp2a.lo.s32.s32 %0, %1, %2, %3;" : "=r"(d) : "r"(a), "r"(b), "r"(c));
+    return d;
+}
+__device__ __forceinline__ int dp2a_hi_ss(uint32_t a, uint32_t b, int c) {
+    int d;
+    asm("dp2a.hi.s32.s32 %0, %1, %2, %3;" : "=r"(d) : "r"(a), "r"(b), "r"(c));
+    return d;
+}
+__device__ __forceinline__ int dp2a_lo_su(uint32_t a, uint32_t b, int c) {
+    int d;
+    asm("dp2a.lo.s32.u32 %0, %1, %2, %3;" : "=r"(d) : "r"(a), "r"(b), "r"(c));
+    return d;
+}
+__device__ __forceinline__ int dp2a_hi_su(uint32_t a, uint32_t b, int c) {
+    int d;
+    asm("dp2a.hi.s32.u32 %0, %1, %2, %3;" : "=r"(d) : "r"(a), "r"(b), "r"(c));
+    return d;
+}
+
+// Position of key (i mod 16) inside its chunk's int16 array, so that the
+// int16 pairs line up with the bytes dp2a reads: natural order for 8 and 6
+// bits; for 4 bits a word's low nibbles hold the even codes of 8 keys and
+// its high nibbles the odd ones.
+template <int BITS>
+__host__ __device__ constexpr int xslot(int r) {
+    if (BITS != 4) return r;
+    const int q = r >> 3, w = r & 7;
+    return 8 * q + ((w & 1) ? 4 + (w >> 1) : (w >> 1));
+}
+
+// One 16-code group as raw words (4 words for 8 bits, 3 for 6 bits, 2 for 4).
+template <int BITS>
+struct Group {
+    uint32_t w[BITS == 8 ? 4 : (BITS == 6 ? 3 : 2)];
+};
+
+template <int BITS>
+__device__ __forceinline__ void load_group(Group<BITS> &g, const uint8_t *p) {
+    if constexpr (BITS == 8) {
+        const uint4 v = __ldcs(reinterpret_cast<const uint4 *>(p));
+        g.w[0] = v.x; g.w[1] = v.y; g.w[2] = v.z; g.w[3] = v.w;
+    } else if constexpr (BITS == 4) {
+        const uint2 v = __ldcs(reinterpret_cast<const uint2 *>(p));
+        g.w[0] = v.x; g.w[1] = v.y;
+    } else {
+        const uint32_t *q = reinterpret_cast<const uint32_t *>(p);
+        g.w[0] = __ldcs(q); g.w[1] = __ldcs(q + 1); g.w[2] = __ldcs(q + 2);
+    }
+}
+
+// Integer dot products of one 16-code group with the int16 chunk of x_k
+// (Xk, 8 words) and x_q (Xq).  For 4 and 6 bits the codes are read as
+// unsigned offset values (code + 8, code + 32); the caller removes
+// bias * sum(X).
+template <int BITS>
+__device__ __forceinline__ void group_dot(const Group<BITS> &g, const uint32_t (&Xk)[8],
+                                          const uint32_t (&Xq)[8], int &ak, int &aq) {
+    if constexpr (BITS == 8) {
+#pragma unroll
+        for (int q = 0; q < 4; ++q) {
+            ak = dp2a_lo_ss(Xk[2 * q], g.w[q], ak);
+            ak = dp2a_hi_ss(Xk[2 * q + 1], g.w[q], ak);
+            aq = dp2a_lo_ss(Xq[2 * q], g.w[q], aq);
+            aq = dp2a_hi_ss(Xq[2 * q + 1], g.w[q], aq);
+        }
+    } else if constexpr (BITS == 4) {
+#pragma unroll
+        for (int q = 0; q < 2; ++q) {
+            const uint32_t lo = (g.w[q] & 0x0F0F0F0Fu) ^ 0x08080808u;         // codes 8q + 0,2,4,6
+            const uint32_t hi = ((g.w[q] >> 4) & 0x0F0F0F0Fu) ^ 0x08080808u;  // codes 8q + 1,3,5,7
+            ak = dp2a_lo_su(Xk[4 * q], lo, ak);
+            ak = dp2a_hi_su(Xk[4 * q + 1], lo, ak);
+            ak = dp2a_lo_su(Xk[4 * q + 2], hi, ak);
+            ak = dp2a_hi_su(Xk[4 * q + 3], hi, ak);
+            aq = dp2a_lo_su(Xq[4 * q], lo, aq);
+            aq = dp2a_hi_su(Xq[4 * q + 1], lo, aq);
+            aq = dp2a_lo_su(Xq[4 * q + 2], hi, aq);
+            aq = dp2a_hi_su(Xq[4 * q + 3], hi, aq);
+        }
+    } else {
+        const uint32_t w0 = g.w[0], w1 = g.w[1], w2 = g.w[2];
+        const uint32_t l[4] = {(w0 & 0x3F3F3F3Fu) ^ 0x20202020u, (w1 & 0x3F3F3F3Fu) ^ 0x20202020u,
+                               (w2 & 0x3F3F3F3Fu) ^ 0x20202020u,
+                               (((w0 >> 6) & 0x03030303u) | ((w1 >> 4) & 0x0C0C0C0Cu) |
+                                ((w2 >> 2) & 0x30303030u)) ^ 0x20202020u};
+#pragma unroll
+        for (int q = 0; q < 4; ++q) {
+            ak = dp2a_lo_su(Xk[2 * q], l[q], ak);
+            ak = dp2a_hi_su(Xk[2 * q + 1], l[q], ak);
+            aq = dp2a_lo_su(Xq[2 * q], l[q], aq);
+            aq = dp2a_hi_su(Xq[2 * q + 1], l[q], aq);
+        }
+    }
+}
+
+// Reduce-scatter of N float2 values over N consecutive lanes of an aligned
 // group (N a power of two <= 32): afterwards lane l holds the group sum of
 // value (l mod N) in v[0].
 template <int N>
-__device__ __forceinline__ void reduce_scatter_group(float (&v)[N], int lane) {
+__device__ __forceinline__ void reduce_scatter2(float2 (&v)[N], int lane) {
 #pragma unroll
     for (int off = N / 2; off >= 1; off >>= 1) {
         const bool upper = (lane & off) != 0;
 #pragma unroll
         for (int i = 0; i < off; ++i) {
-            const float send = upper ? v[i] : v[i + off];
-            const float keep = upper ? v[i + off] : v[i];
-            v[i] = keep + __shfl_xor_sync(0xFFFFFFFFu, send, off);
+            const float2 send = upper ? v[i] : v[i + off];
+            const float2 keep = upper ? v[i + off] : v[i];
+            v[i].x = keep.x + __shfl_xor_sync(0xFFFFFFFFu, send.x, off);
+            v[i].y = keep.y + __shfl_xor_sync(0xFFFFFFFFu, send.y, off);
         }
     }
 }
@@ -74,229 +236,338 @@ __device__ __forceinline__ float warp_sum(float x) {
 }
 
 template <int D, int BITS>
-__global__ void __launch_bounds__(2 * D) decode_kernel(DecodeArgs A) {
-    constexpr int NT = 2 * D, CPR = D / 16, MR = D / 32, E = D / 32;
+__global__ void __launch_bounds__(D + 32) decode_kernel(DecodeArgs A) {
+    constexpr int NC = D;            // consumer threads
+    constexpr int LPR = D / 16;      // threads per row, one 16-key chunk each
+    constexpr int RPT = D / 16;      // rows per thread (16 row groups)
     constexpr int GB = group_bytes<BITS>();
-    static_assert(2 * MR == CPR, "one value per lane after the reduce-scatter");
+    constexpr int NCH = D / 16;      // chunks per row
+    constexpr int KPL = D / 16;      // keys per thread in the dot-product phase
+    constexpr int NJ = NC / 16;      // dot-product jobs per pass
+    constexpr int BIAS = BITS == 8 ? 0 : (BITS == 6 ? 32 : 8);
     const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
-    const size_t head = blockIdx.x;
-    const Layout &L = A.L;
-    const Flags &F = A.F;
-    uint8_t *blob = A.state + head * L.blob;
+    const Layout L = A.L;
+    const Flags F = A.F;
+    const DecodeStage SG = decode_stage(L, D, F.window, F.bf16_in, F.kda);
+    const int G = gridDim.x;
+    const int n_mine = (A.num_heads - (int)blockIdx.x + G - 1) / G;
 
     extern __shared__ __align__(128) uint8_t smem[];
-    uint64_t *bar = reinterpret_cast<uint64_t *>(smem);
-    uint32_t *s_hdr = reinterpret_cast<uint32_t *>(smem + 16);  // count, status, ncomp, skip, g, newbits
-    uint32_t *s_meta = reinterpret_cast<uint32_t *>(smem + 64);
-    float *s_y = reinterpret_cast<float *>(smem + 128);  // y_k [D] | y_q [D]
-    float *s_x = s_y + 2 * D;                            // x_k [D] | x_q [D]
-    float *s_gemv = s_x + 2 * D;                         // R^T y_k [D] | R^T y_q [D] (before qs)
-    float *s_dot = s_gemv + 2 * D;                       // k-side [kDotSlots] | q-side
-    float *s_red = s_dot + 2 * kDotSlots;                // [32]
-    uint8_t *s_cmp = smem + decode_fixed_smem<D>();      // qs | sm | comp_vec | codes
-    float *s_pairs = reinterpret_cast<float *>(s_cmp + align_up(L.compact_bytes, 128));
-    const uint8_t *s_qs = s_cmp;
-    const uint8_t *s_sm = s_cmp + (L.sm_off - L.qs_off);
-    const float *s_cvec = reinterpret_cast<const float *>(s_cmp + (L.cvec_off - L.qs_off));
-    const uint8_t *s_codes = s_cmp + (L.codes_off - L.qs_off);
+    uint64_t *full = reinterpret_cast<uint64_t *>(smem);  // [2]
+    uint64_t *empty = full + 2;                           // [2]
+    volatile uint32_t *s_abort = reinterpret_cast<volatile uint32_t *>(smem + 120);
+    float *s_y = reinterpret_cast<float *>(smem + 128);          // y_k [D] | y_q [D]
+    int16_t *s_X = reinterpret_cast<int16_t *>(s_y + 2 * D);     // X_k [D] | X_q [D] (chunk order)
+    float *s_sc = reinterpret_cast<float *>(s_X + 2 * D);        // chunk scales k [NCH] | q [NCH]
+    float *s_dot = s_sc + 2 * NCH;                               // k-side [kDotSlots] | q-side
+    float *s_cadd = s_dot + 2 * kDotSlots;                       // column-compensator terms [2][D]
+    float *s_kh = s_cadd + 2 * D;                                // new key, window-start frame [D]
+    float *s_g = s_kh + D;                                       // new decay product [D]
+    float *s_red = s_g + D;                                      // [32]
+    uint32_t *s_cnt = reinterpret_cast<uint32_t *>(s_red + 32);  // producer batch [32]
+    float *s_pbeta = reinterpret_cast<float *>(s_cnt + 32);
+    float *s_palpha = s_pbeta + 32;
+    uint32_t *s_rowc = reinterpret_cast<uint32_t *>(s_palpha + 32);  // key-row compensators [16]
+    uint32_t *s_colc = s_rowc + 16;                                  // value-column compensators [16]
+    uint32_t *s_info = s_colc + 16;                                  // run, count, nrow, ncol, newbits
+    uint8_t *stages = smem + decode_fixed_smem<D>();
 
     if (tid == 0) {
-        mbar_init(&bar[0], 1);
-        mbar_init(&bar[1], 1);
-        fence_mbar_init();
-        mbar_arrive_expect_tx(&bar[0], L.compact_bytes);
-        bulk_g2s(s_cmp, blob + L.qs_off, L.compact_bytes, &bar[0]);
-        const uint4 h = *reinterpret_cast<const uint4 *>(blob);  // count, status, ncomp, magic
-        const uint32_t g_bits = *reinterpret_cast<const uint32_t *>(blob + kHdrG);
-        const uint4 *gm = reinterpret_cast<const uint4 *>(blob + kHdrMeta);
-        uint4 *sm4 = reinterpret_cast<uint4 *>(s_meta);
-#pragma unroll
-        for (int x = 0; x < 4; ++x) sm4[x] = gm[x];
-        bool meta_ok = true;
-        for (uint32_t cc = 0; cc < h.z && cc < (uint32_t)kMaxComp; ++cc)
-            meta_ok &= (s_meta[cc] & 0x7FFFFFFFu) < (uint32_t)D;
-        uint32_t newbits = 0;
-        if (h.w != kMagic || h.z > (uint32_t)F.num_comp || h.x > (uint32_t)F.window || !meta_ok)
-            newbits = LQ_DEV_CORRUPT;
-        else if (h.y == 0 && h.x >= (uint32_t)F.window)
-            newbits = LQ_DEV_WINDOW_FULL;
-        const bool run = h.y == 0 && newbits == 0;
-        const uint32_t pbytes = run ? h.x * L.pair_bytes : 0u;
-        mbar_arrive_expect_tx(&bar[1], pbytes);
-        if (pbytes) bulk_g2s(s_pairs, blob + L.pairs_off, pbytes, &bar[1]);
-        s_hdr[0] = h.x;
-        s_hdr[1] = h.y;
-        s_hdr[2] = h.z;
-        s_hdr[3] = run ? 0u : 1u;
-        s_hdr[4] = g_bits;
-        s_hdr[5] = newbits;
-    }
-
-    // inputs of this token (independent of the state)
-    float kv = 0.f, qv = 0.f, vv = 0.f, av = 1.f, gold = 1.f;
-    if (tid < D) {
-        const size_t o = head * D + tid;
-        kv = load_in(A.k, o, F.bf16_in);
-        qv = load_in(A.q, o, F.bf16_in);
-        vv = load_in(A.v, o, F.bf16_in);
-        if (F.kda) {
-            av = A.decay[o];
-            gold = reinterpret_cast<const float *>(blob + L.g_off)[tid];
+        for (int s = 0; s < kDecodeStages; ++s) {
+            mbar_init(&full[s], 1);
+            mbar_init(&empty[s], 1);
         }
+        *s_abort = 0u;
+        fence_mbar_init();
     }
-    const float bt = A.beta[head];
-    const float alpha = F.kda ? 1.f : A.decay[head];
     __syncthreads();
 
-    uint32_t skip = s_hdr[3];
-    const uint32_t count = s_hdr[0], ncomp = s_hdr[2];
-    if (!F.kda) {
-        gold = __uint_as_float(s_hdr[4]);
-        av = alpha;
-    }
-    const float gnew = gold * av;
-    const bool bad = (tid < D) && !(gnew >= kMinDecayProduct);
-    const int any_bad = __syncthreads_or(bad);
-    uint32_t newbits = s_hdr[5];
-    if (!skip && any_bad) {
-        skip = 1;
-        newbits = LQ_DEV_RANGE;
-    }
-
-    bool ok = true;
-    if (!skip) {
-        if (tid < D) {
-            s_y[tid] = gnew * kv;
-            s_y[D + tid] = gnew * qv;
+    if (warp == NC / 32) {
+        // ------------------------------------------------ producer warp
+        for (int base = 0; base < n_mine; base += 32) {
+            const int i = base + lane;
+            if (i < n_mine) {
+                const size_t h = blockIdx.x + (size_t)i * G;
+                s_cnt[lane] = *reinterpret_cast<const uint32_t *>(A.state + h * L.blob + kHdrCount);
+                s_pbeta[lane] = A.beta[h];
+                s_palpha[lane] = F.kda ? 1.f : A.decay[h];
+            }
+            __syncwarp();
+            if (lane == 0) {
+                const int nb = min(32, n_mine - base);
+                for (int x = 0; x < nb && !*s_abort; ++x) {
+                    const int it = base + x, s = it % kDecodeStages;
+                    if (it >= kDecodeStages && !mbar_wait_bounded(&empty[s], ((it / kDecodeStages) - 1) & 1)) {
+                        *s_abort = 1u;
+                        break;
+                    }
+                    const size_t h = blockIdx.x + (size_t)it * G;
+                    const uint8_t *blob = A.state + h * L.blob;
+                    uint8_t *st = stages + (size_t)s * SG.bytes;
+                    const uint32_t c = s_cnt[x];
+                    const uint32_t cc = c < (uint32_t)F.window ? c : 0u;
+                    float *aux = reinterpret_cast<float *>(st + SG.aux_off);
+                    aux[0] = s_pbeta[x];
+                    aux[1] = s_palpha[x];
+                    const uint32_t pb = cc * L.pair_bytes;
+                    mbar_arrive_expect_tx(&full[s], L.codes_off + pb + 3 * SG.qkv_bytes +
+                                                        (F.kda ? (uint32_t)D * 4u : 0u));
+                    bulk_g2s(st, blob, L.codes_off, &full[s]);
+                    if (pb) bulk_g2s(st + SG.pairs_at, blob + L.pairs_off, pb, &full[s]);
+                    const size_t qo = h * (size_t)SG.qkv_bytes;
+                    bulk_g2s(st + SG.in_off, static_cast<const uint8_t *>(A.q) + qo, SG.qkv_bytes, &full[s]);
+                    bulk_g2s(st + SG.in_off + SG.qkv_bytes, static_cast<const uint8_t *>(A.k) + qo,
+                             SG.qkv_bytes, &full[s]);
+                    bulk_g2s(st + SG.in_off + 2 * SG.qkv_bytes, static_cast<const uint8_t *>(A.v) + qo,
+                             SG.qkv_bytes, &full[s]);
+                    if (F.kda) bulk_g2s(st + SG.dec_off, A.decay + h * D, (uint32_t)D * 4u, &full[s]);
+                }
+            }
+            __syncwarp();
         }
-        float kq = (tid < D) ? kv * qv : 0.f;
-        kq = warp_sum(kq);
-        if (lane == 0) s_red[warp] = kq;
-        ok = __syncthreads_and(mbar_wait_bounded(&bar[0], 0));
-        if (ok) {
-            if (tid < D) {
-                const float smv = load_scale(s_sm, tid, F.f16_scale);
-                s_x[tid] = smv * s_y[tid];
-                s_x[D + tid] = smv * s_y[D + tid];
-            }
-            __syncthreads();
+        return;
+    }
 
-            // ---- fused dequantize + dual GEMV over the codes
-            const int c = tid % CPR, rg = tid / CPR;
-            float xk[16], xq[16];
+    // ---------------------------------------------------- consumer threads
+    // GEMV role: chunk c of rows j = RPT*rg + m (m < RPT); after the
+    // reduce-scatter this thread owns row jrow = RPT*rg + c, so a warp's rows
+    // are 32 consecutive value channels.
+    const int c = tid % LPR, rg = tid / LPR;
+    const int jrow = RPT * rg + c;
+    // dot-product role: job slot and key chunk
+    const int djob = tid / 16, dkc = tid % 16;
+    const uint8_t *code_base = A.state + L.codes_off + c * GB;
+
+    Group<BITS> cg[RPT];
+    if (n_mine > 0) {
+        const uint8_t *cb = code_base + (size_t)blockIdx.x * L.blob;
 #pragma unroll
-            for (int x = 0; x < 16; x += 4) {
-                const float4 a4 = *reinterpret_cast<const float4 *>(s_x + 16 * c + x);
-                const float4 b4 = *reinterpret_cast<const float4 *>(s_x + D + 16 * c + x);
-                xk[x] = a4.x; xk[x + 1] = a4.y; xk[x + 2] = a4.z; xk[x + 3] = a4.w;
-                xq[x] = b4.x; xq[x + 1] = b4.y; xq[x + 2] = b4.z; xq[x + 3] = b4.w;
+        for (int m = 0; m < RPT; ++m) load_group<BITS>(cg[m], cb + (size_t)(RPT * rg + m) * L.row_bytes);
+    }
+
+    for (int it = 0; it < n_mine; ++it) {
+        const int s = it % kDecodeStages;
+        const uint32_t ph = (uint32_t)(it / kDecodeStages) & 1u;
+        const uint8_t *st = stages + (size_t)s * SG.bytes;
+        const size_t h = blockIdx.x + (size_t)it * G;
+        uint8_t *blob = A.state + h * L.blob;
+        const bool has_next = it + 1 < n_mine;
+        const uint8_t *next_codes = code_base + (h + G) * (size_t)L.blob;
+        if (!consumer_sync_and(mbar_wait_bounded(&full[s], ph), NC)) {
+            // the copy never completed: record it on this blob and stop this CTA
+            if (tid == 0) {
+                set_status(blob, LQ_DEV_TIMEOUT);
+                *s_abort = 1u;
             }
-            float acc[2 * MR];
-#pragma unroll
-            for (int m = 0; m < MR; ++m) {
-                const int j = rg + 32 * m;
-                float cf[16];
-                unpack16<BITS>(s_codes + (size_t)j * L.row_bytes + c * GB, cf);
-                float ak = 0.f, aq = 0.f;
-#pragma unroll
-                for (int x = 0; x < 16; ++x) {
-                    ak = fmaf(cf[x], xk[x], ak);
-                    aq = fmaf(cf[x], xq[x], aq);
-                }
-                acc[m] = ak;
-                acc[MR + m] = aq;
-            }
-            reduce_scatter_group<CPR>(acc, lane);
-            {
-                const int idx = lane & (CPR - 1);
-                const int side = idx / MR, m = idx % MR;
-                s_gemv[side * D + rg + 32 * m] = acc[0];
-            }
-            ok = __syncthreads_and(mbar_wait_bounded(&bar[1], 0));
+            A.out[h * D + tid] = 0.f;
+            break;
         }
-        if (ok) {
-            // ---- dot products of buffered keys and compensator columns with y
-            float yk[E], yq[E];
-#pragma unroll
-            for (int e = 0; e < E; ++e) {
-                yk[e] = s_y[lane * E + e];
-                yq[e] = s_y[D + lane * E + e];
-            }
-            const int jobs = (int)(count + ncomp);
-            for (int jb = warp; jb < jobs; jb += NT / 32) {
-                const float *vec;
-                if (jb < (int)count) {
-                    vec = s_pairs + (size_t)jb * 2 * D;
-                } else {
-                    const uint32_t meta = s_meta[jb - count];
-                    if (!(meta & kCompCol)) continue;  // key-row lines need no dot
-                    vec = s_cvec + (size_t)(jb - count) * D;
-                }
-                float dk_ = 0.f, dq_ = 0.f;
-#pragma unroll
-                for (int e = 0; e < E; ++e) {
-                    const float x = vec[lane * E + e];
-                    dk_ = fmaf(x, yk[e], dk_);
-                    dq_ = fmaf(x, yq[e], dq_);
-                }
-                dk_ = warp_sum(dk_);
-                dq_ = warp_sum(dq_);
-                if (lane == 0) {
-                    s_dot[jb] = dk_;
-                    s_dot[kDotSlots + jb] = dq_;
-                }
-            }
-            __syncthreads();
+        const float *aux = reinterpret_cast<const float *>(st + SG.aux_off);
+        const uint8_t *qkv = st + SG.in_off;
 
-            // ---- combine, delta update, output, append the pair
-            if (tid < D) {
-                const int j = tid;
-                float kq = 0.f;
+        if (warp == 0) {
+            // header checks and compensator lists (one warp, ballots)
+            const uint4 hdr = *reinterpret_cast<const uint4 *>(st);  // count, status, ncomp, magic
+            const uint32_t ncomp = hdr.z;
+            const bool inl = lane < (int)min(ncomp, (uint32_t)kMaxComp);
+            const uint32_t m = inl ? reinterpret_cast<const uint32_t *>(st + kHdrMeta)[lane] : 0u;
+            const bool iscol = inl && (m & kCompCol), isrow = inl && !(m & kCompCol);
+            const unsigned colm = __ballot_sync(0xFFFFFFFFu, iscol);
+            const unsigned rowm = __ballot_sync(0xFFFFFFFFu, isrow);
+            const unsigned badm = __ballot_sync(0xFFFFFFFFu, inl && (m & 0x7FFFFFFFu) >= (uint32_t)D);
+            const unsigned lt = (1u << lane) - 1u;
+            if (iscol) s_colc[__popc(colm & lt)] = (uint32_t)lane;
+            if (isrow) s_rowc[__popc(rowm & lt)] = (uint32_t)lane;
+            if (lane == 0) {
+                uint32_t newbits = 0;
+                if (hdr.w != kMagic || ncomp > (uint32_t)F.num_comp || hdr.x > (uint32_t)F.window || badm)
+                    newbits = LQ_DEV_CORRUPT;
+                else if (hdr.y == 0 && hdr.x >= (uint32_t)F.window)
+                    newbits = LQ_DEV_WINDOW_FULL;
+                s_info[0] = (hdr.y == 0 && newbits == 0) ? 1u : 0u;
+                s_info[1] = hdr.x;
+                s_info[2] = (uint32_t)__popc(rowm);
+                s_info[3] = (uint32_t)__popc(colm);
+                s_info[4] = newbits;
+            }
+        }
+        bool bad;
+        {
+            const int i = tid;
+            const float kv = load_in(qkv + SG.qkv_bytes, i, F.bf16_in);
+            const float qv = load_in(qkv, i, F.bf16_in);
+            float a, gold;
+            if (F.kda) {
+                a = reinterpret_cast<const float *>(st + SG.dec_off)[i];
+                gold = reinterpret_cast<const float *>(st + L.g_off)[i];
+            } else {
+                a = aux[1];
+                gold = *reinterpret_cast<const float *>(st + kHdrG);
+            }
+            const float gnew = gold * a;
+            bad = !(gnew >= kMinDecayProduct);
+            const float yk = gnew * kv, yq = gnew * qv;
+            s_y[i] = yk;
+            s_y[D + i] = yq;
+            s_kh[i] = bad ? 0.f : __fdiv_rn(kv, gnew);  // the new key in the window-start frame
+            s_g[i] = gnew;
+            s_cadd[i] = 0.f;
+            s_cadd[D + i] = 0.f;
+            // x = sm . y, quantized per 16-key chunk to int16 with the chunk's scale
+            const float smv = load_scale(st + L.sm_off, i, F.f16_scale);
+            const float xk = smv * yk, xq = smv * yq;
+            float mk = fabsf(xk), mq = fabsf(xq);
 #pragma unroll
-                for (int w = 0; w < D / 32; ++w) kq += s_red[w];
-                const float qsj = load_scale(s_qs, j, F.f16_scale);
-                float a = qsj * s_gemv[j];
-                float b = qsj * s_gemv[D + j];
-                for (uint32_t cc = 0; cc < ncomp; ++cc) {
-                    const uint32_t meta = s_meta[cc];
-                    if (meta & kCompCol) {
-                        if ((int)(meta & 0x7FFFFFFFu) == j) {
-                            a += s_dot[count + cc];
-                            b += s_dot[kDotSlots + count + cc];
+            for (int off = 8; off >= 1; off >>= 1) {
+                mk = fmaxf(mk, __shfl_xor_sync(0xFFFFFFFFu, mk, off));
+                mq = fmaxf(mq, __shfl_xor_sync(0xFFFFFFFFu, mq, off));
+            }
+            const float ik = mk > 0.f ? 32767.f / mk : 0.f, iq = mq > 0.f ? 32767.f / mq : 0.f;
+            const int slot = (i & ~15) + xslot<BITS>(i & 15);
+            s_X[slot] = (int16_t)max(-32767, min(32767, __float2int_rn(xk * ik)));
+            s_X[D + slot] = (int16_t)max(-32767, min(32767, __float2int_rn(xq * iq)));
+            if ((i & 15) == 0) {
+                s_sc[i >> 4] = ik > 0.f ? 1.f / ik : 0.f;
+                s_sc[NCH + (i >> 4)] = iq > 0.f ? 1.f / iq : 0.f;
+            }
+            const float kq = warp_sum(kv * qv);
+            if (lane == 0) s_red[warp] = kq;
+        }
+        const bool any_bad = consumer_sync_or(bad, NC);
+        bool run = s_info[0] != 0u;
+        const uint32_t count = s_info[1];
+        const int nrow = (int)s_info[2], ncol = (int)s_info[3];
+        uint32_t newbits = s_info[4];
+        if (run && any_bad) {
+            run = false;
+            newbits = LQ_DEV_RANGE;
+        }
+
+        if (run) {
+            const float *pairs = reinterpret_cast<const float *>(st + SG.pairs_at);
+            const float *cvec = reinterpret_cast<const float *>(st + L.cvec_off);
+            const uint32_t *meta = reinterpret_cast<const uint32_t *>(st + kHdrMeta);
+            // ---- dot products of buffered keys / compensator columns with y
+            const int jobs = (int)count + ncol;
+            if (jobs > 0) {
+                float yk[KPL], yq[KPL];
+#pragma unroll
+                for (int e = 0; e < KPL; e += 4) {
+                    const float4 a4 = *reinterpret_cast<const float4 *>(s_y + dkc * KPL + e);
+                    const float4 b4 = *reinterpret_cast<const float4 *>(s_y + D + dkc * KPL + e);
+                    yk[e] = a4.x; yk[e + 1] = a4.y; yk[e + 2] = a4.z; yk[e + 3] = a4.w;
+                    yq[e] = b4.x; yq[e + 1] = b4.y; yq[e + 2] = b4.z; yq[e + 3] = b4.w;
+                }
+                for (int jb0 = 0; jb0 < jobs; jb0 += NJ) {
+                    const int jb = jb0 + djob;
+                    const bool live = jb < jobs;
+                    float dk_ = 0.f, dq_ = 0.f;
+                    if (live) {
+                        const float *vec = jb < (int)count ? pairs + (size_t)jb * 2 * D
+                                                           : cvec + (size_t)s_colc[jb - count] * D;
+#pragma unroll
+                        for (int e = 0; e < KPL; e += 4) {
+                            const float4 x4 = *reinterpret_cast<const float4 *>(vec + dkc * KPL + e);
+                            dk_ = fmaf(x4.x, yk[e], dk_); dk_ = fmaf(x4.y, yk[e + 1], dk_);
+                            dk_ = fmaf(x4.z, yk[e + 2], dk_); dk_ = fmaf(x4.w, yk[e + 3], dk_);
+                            dq_ = fmaf(x4.x, yq[e], dq_); dq_ = fmaf(x4.y, yq[e + 1], dq_);
+                            dq_ = fmaf(x4.z, yq[e + 2], dq_); dq_ = fmaf(x4.w, yq[e + 3], dq_);
                         }
-                    } else {
-                        const float wj = s_cvec[(size_t)cc * D + j];
-                        a = fmaf(s_y[meta], wj, a);
-                        b = fmaf(s_y[D + meta], wj, b);
+                    }
+#pragma unroll
+                    for (int off = 8; off >= 1; off >>= 1) {
+                        dk_ += __shfl_xor_sync(0xFFFFFFFFu, dk_, off);
+                        dq_ += __shfl_xor_sync(0xFFFFFFFFu, dq_, off);
+                    }
+                    if (live && dkc == 0) {
+                        if (jb < (int)count) {
+                            s_dot[jb] = dk_;
+                            s_dot[kDotSlots + jb] = dq_;
+                        } else {
+                            const int j0 = (int)(meta[s_colc[jb - count]] & 0x7FFFFFFFu);
+                            s_cadd[j0] = dk_;
+                            s_cadd[D + j0] = dq_;
+                        }
                     }
                 }
-                for (uint32_t m = 0; m < count; ++m) {
-                    const float uj = s_pairs[(size_t)m * 2 * D + D + j];
-                    a = fmaf(s_dot[m], uj, a);
-                    b = fmaf(s_dot[kDotSlots + m], uj, b);
-                }
-                const float u = bt * (vv - a);
-                A.out[head * D + j] = fmaf(kq, u, b);
-                float *pair = reinterpret_cast<float *>(blob + L.pairs_off + (size_t)count * L.pair_bytes);
-                pair[j] = __fdiv_rn(kv, gnew);  // key j in the window-start frame
-                pair[D + j] = u;
-                if (F.kda) reinterpret_cast<float *>(blob + L.g_off)[j] = gnew;
             }
+            consumer_sync(NC);
+
+            // ---- fused dequantize + dual GEMV over the codes (integer pipe)
+            uint32_t Xk[8], Xq[8];
+            {
+                const uint4 *xk4 = reinterpret_cast<const uint4 *>(s_X + 16 * c);
+                const uint4 *xq4 = reinterpret_cast<const uint4 *>(s_X + D + 16 * c);
+                const uint4 a0 = xk4[0], a1 = xk4[1], b0 = xq4[0], b1 = xq4[1];
+                Xk[0] = a0.x; Xk[1] = a0.y; Xk[2] = a0.z; Xk[3] = a0.w;
+                Xk[4] = a1.x; Xk[5] = a1.y; Xk[6] = a1.z; Xk[7] = a1.w;
+                Xq[0] = b0.x; Xq[1] = b0.y; Xq[2] = b0.z; Xq[3] = b0.w;
+                Xq[4] = b1.x; Xq[5] = b1.y; Xq[6] = b1.z; Xq[7] = b1.w;
+            }
+            const float sck = s_sc[c], scq = s_sc[NCH + c];
+            int biask = 0, biasq = 0;
+            if constexpr (BIAS != 0) {
+#pragma unroll
+                for (int x = 0; x < 8; ++x) {  // sum of the chunk's 16 entries
+                    biask = dp2a_lo_ss(Xk[x], 0x00000101u, biask);
+                    biasq = dp2a_lo_ss(Xq[x], 0x00000101u, biasq);
+                }
+                biask *= BIAS;
+                biasq *= BIAS;
+            }
+            float2 acc[RPT];
+#pragma unroll
+            for (int m = 0; m < RPT; ++m) {
+                int ak = -biask, aq = -biasq;
+                group_dot<BITS>(cg[m], Xk, Xq, ak, aq);
+                if (has_next) load_group<BITS>(cg[m], next_codes + (size_t)(RPT * rg + m) * L.row_bytes);
+                acc[m] = make_float2((float)ak * sck, (float)aq * scq);
+            }
+            reduce_scatter2<LPR>(acc, lane);
+
+            // ---- epilogue: this thread owns (a_j, b_j) of row j
+            const int j = jrow;
+            const float qsj = load_scale(st + L.qs_off, j, F.f16_scale);
+            float a = qsj * acc[0].x + s_cadd[j];
+            float b = qsj * acc[0].y + s_cadd[D + j];
+            for (int r = 0; r < nrow; ++r) {
+                const uint32_t cc = s_rowc[r];
+                const float wj = cvec[(size_t)cc * D + j];
+                const int i0 = (int)(meta[cc] & 0x7FFFFFFFu);
+                a = fmaf(s_y[i0], wj, a);
+                b = fmaf(s_y[D + i0], wj, b);
+            }
+            const float *up = pairs + D + j;
+#pragma unroll 4
+            for (uint32_t m = 0; m < count; ++m) {
+                const float uj = up[(size_t)m * 2 * D];
+                a = fmaf(s_dot[m], uj, a);
+                b = fmaf(s_dot[kDotSlots + m], uj, b);
+            }
+            const float u = aux[0] * (load_in(qkv + 2 * SG.qkv_bytes, j, F.bf16_in) - a);
+            float kq = 0.f;
+#pragma unroll
+            for (int w = 0; w < NC / 32; ++w) kq += s_red[w];
+            A.out[h * D + j] = fmaf(kq, u, b);
+            float *pair = reinterpret_cast<float *>(blob + L.pairs_off + (size_t)count * L.pair_bytes);
+            pair[D + j] = u;
+            pair[tid] = s_kh[tid];
+            if (F.kda) reinterpret_cast<float *>(blob + L.g_off)[tid] = s_g[tid];
             if (tid == 0) {
                 *reinterpret_cast<uint32_t *>(blob + kHdrCount) = count + 1;
-                if (!F.kda) *reinterpret_cast<float *>(blob + kHdrG) = gnew;
+                if (!F.kda) *reinterpret_cast<float *>(blob + kHdrG) = s_g[0];
             }
-            return;
+        } else {
+            // skipped: still move on to the next blob's codes
+            if (has_next) {
+#pragma unroll
+                for (int m = 0; m < RPT; ++m) load_group<BITS>(cg[m], next_codes + (size_t)(RPT * rg + m) * L.row_bytes);
+            }
+            A.out[h * D + tid] = 0.f;
+            if (tid == 0 && newbits) set_status(blob, newbits);
         }
-        newbits = LQ_DEV_TIMEOUT;
-    }
-
-    // skipped (or a copy wait timed out): zero output, record, drain copies
-    if (tid < D) A.out[head * D + tid] = 0.f;
-    if (tid == 0) {
-        if (newbits) set_status(blob, newbits);
-        mbar_wait_bounded(&bar[0], 0);
-        mbar_wait_bounded(&bar[1], 0);
+        consumer_sync(NC);  // every consumer is done with stage s and the scratch
+        if (tid == 0) mbar_arrive(&empty[s]);
     }
 }
 
