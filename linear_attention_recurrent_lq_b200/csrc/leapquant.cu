@@ -107,8 +107,19 @@ lq_status launch_decode(const lq_config &c, const DecodeArgs &a, cudaStream_t s)
 
 template <int D, int BITS, int MODE>
 lq_status launch_boundary(const lq_config &c, const FlushArgs &a, cudaStream_t s) {
-    const uint32_t smem = flush_smem_bytes(D, BITS, a.L, c.window, c.decay_kind);
-    auto k = boundary_kernel<D, BITS, MODE>;
+    if (MODE == 0) {  // persistent flush
+        const uint32_t smem = flush_smem_bytes(D, BITS, a.L, c.window);
+        auto k = flush_kernel<D, BITS>;
+        cudaError_t e = allow_smem(k, smem);
+        if (e != cudaSuccess) return LQ_ERR_CUDA;
+        const int threads = 4 * D + 32;
+        const int grid = persistent_grid(k, threads, smem, a.num_heads);
+        if (grid <= 0) return LQ_ERR_CUDA;
+        k<<<grid, threads, smem, s>>>(a);
+        return launched(cudaSuccess);
+    }
+    const uint32_t smem = boundary_smem_bytes(D, BITS, a.L, c.window);
+    auto k = boundary_kernel<D, BITS, MODE == 0 ? 1 : MODE>;
     cudaError_t e = allow_smem(k, smem);
     if (e != cudaSuccess) return LQ_ERR_CUDA;
     k<<<(unsigned)(c.num_slots * c.num_heads), 4 * D, smem, s>>>(a);
@@ -174,7 +185,7 @@ lq_status lq_state_init(const lq_config *cfg, void *state, const float *S0, lq_s
         a.L = L;
         return launch_fp32_copy<1>(c, a, s);
     }
-    FlushArgs a{static_cast<uint8_t *>(state), S0, nullptr, L, make_flags(c)};
+    FlushArgs a{static_cast<uint8_t *>(state), S0, nullptr, L, make_flags(c), c.num_slots * c.num_heads};
     return dispatch_boundary<1>(c, a, s);
 }
 
@@ -215,7 +226,8 @@ lq_status lq_window_flush(const lq_config *cfg, void *state, lq_stream_t stream)
     if (!aligned(state, 256)) return LQ_ERR_MISALIGNED;
     const lq_config &c = *cfg;
     if (c.bits == 32) return LQ_OK;
-    FlushArgs a{static_cast<uint8_t *>(state), nullptr, nullptr, make_layout(c), make_flags(c)};
+    FlushArgs a{static_cast<uint8_t *>(state), nullptr, nullptr, make_layout(c), make_flags(c),
+                c.num_slots * c.num_heads};
     return dispatch_boundary<0>(c, a, reinterpret_cast<cudaStream_t>(stream));
 }
 
@@ -235,7 +247,7 @@ lq_status lq_dequant_state(const lq_config *cfg, const void *state, float *S_out
         a.L = L;
         return launch_fp32_copy<2>(c, a, s);
     }
-    FlushArgs a{st8, nullptr, S_out, L, make_flags(c)};
+    FlushArgs a{st8, nullptr, S_out, L, make_flags(c), c.num_slots * c.num_heads};
     return dispatch_boundary<2>(c, a, s);
 }
 
