@@ -112,7 +112,7 @@ lq_status launch_boundary(const lq_config &c, const FlushArgs &a, cudaStream_t s
         auto k = flush_kernel<D, BITS>;
         cudaError_t e = allow_smem(k, smem);
         if (e != cudaSuccess) return LQ_ERR_CUDA;
-        const int threads = 4 * D + 32;
+        const int threads = kGroup;
         const int grid = persistent_grid(k, threads, smem, a.num_heads);
         if (grid <= 0) return LQ_ERR_CUDA;
         k<<<grid, threads, smem, s>>>(a);
@@ -122,7 +122,7 @@ lq_status launch_boundary(const lq_config &c, const FlushArgs &a, cudaStream_t s
     auto k = boundary_kernel<D, BITS, MODE == 0 ? 1 : MODE>;
     cudaError_t e = allow_smem(k, smem);
     if (e != cudaSuccess) return LQ_ERR_CUDA;
-    k<<<(unsigned)(c.num_slots * c.num_heads), 4 * D, smem, s>>>(a);
+    k<<<(unsigned)(c.num_slots * c.num_heads), kGroup, smem, s>>>(a);
     return launched(cudaSuccess);
 }
 

@@ -22,37 +22,42 @@
 //    rounded to f16 when stored so), C_ji = clamp(rint(fl32(R'_ij / qs_j))),
 //    ties to even.
 //
-// 4*D consumer threads per (slot, head), each owning a TI x 4 tile of the
-// state (TI = D/16, layout below) in registers through every stage; row and
-// column reductions go through warp shuffles, then across warps through
-// shared memory.  Line energies for the compensator choice are kept in FP64
-// (exact squares), so taking a line can update the other side's energies in
-// place without cancellation trouble.  Every entry
-// of the rebuild follows the rule's operation order exactly (packed FP32x2
-// instructions round each lane like the scalar ones), so the flush compresses
-// the same FP32 matrix lq_dequant_state returns.  The flush kernel is
-// persistent: a producer warp double-buffers each blob (compact state and
-// buffered pairs) into shared memory with bulk async copies, the consumers
-// rebuild from shared memory, release the stage, then compress from registers
-// and write the new compact state straight to global memory.
+// 256 threads handle one (slot, head): each keeps a TI x TJ tile of the
+// state (TI = TJ = D/16) in registers through every stage, as float2 pairs
+// of adjacent key rows so that packed FP32x2 instructions work on register
+// pairs.  Row and column partials go through warp shuffles, then through
+// shared memory; each thread then combines the partials of its own rows and
+// columns, so a scale costs one barrier.  Every entry of the rebuild follows
+// the rule's operation order exactly (packed FP32x2 instructions round each
+// lane like the scalar ones), so the flush compresses the same FP32 matrix
+// lq_dequant_state returns.  Line energies for the compensator choice are
+// FP64 sums of exact squares.  Every warp keeps its own copy of them and runs
+// the same argmax; taking a line lowers the other side's energies in place
+// (no cancellation trouble in FP64), so a round costs one barrier.
+// The flush kernel is persistent, two CTAs per SM, each double-buffering
+// its blobs (compact state and buffered pairs) into shared memory with bulk
+// async copies: the 256 threads rebuild from shared memory, release the
+// stage (one thread refills it with the blob after next), then compress from
+// registers and write the new compact state straight to global memory.
 #pragma once
 
 #include "lq_common.cuh"
 
 namespace lq {
 
-// Thread tiling of a D x D state (NT = 4D threads): warp w owns a
-// (4*TI) x 32 block, rows 4*TI*wi.., columns 32*wj.. (wi = w % WR,
+constexpr int kGroup = 256;  // consumer threads per (slot, head)
+
+// Tiling of a D x D state over the 256 consumers: warp w owns a
+// (4*TI) x (8*TJ) block, rows 4*TI*wi.., columns 8*TJ*wj.. (wi = w % WR,
 // wj = w / WR); lane (li = lane % 4, lj = lane / 4) owns rows
-// i0 = 4*TI*wi + TI*li .. +TI and columns j0 = 32*wj + 4*lj .. +4.  Lanes
-// with the same li read the same key slice of a buffered pair and lanes
-// with the same lj the same value slice, so the rebuild's shared loads are
-// broadcasts.
+// i0 = 4*TI*wi + TI*li .. +TI and columns j0 = 8*TJ*wj + TJ*lj .. +TJ.  Lanes
+// with the same li read the same key slice of a buffered pair and lanes with
+// the same lj the same value slice, so the rebuild's shared loads broadcast.
 template <int D>
 struct FT {
-    static constexpr int NT = 4 * D, TI = D / 16, NW = NT / 32;
-    static constexpr int WR = D / (4 * TI), WC = D / 32;  // warp grid (rows x cols)
-    static_assert(WR * WC == NW, "warp tiling");
+    static constexpr int TI = D / 16, TJ = D / 16, IP = TI / 2;
+    static constexpr int WR = D / (4 * TI), WC = D / (8 * TJ), KE = D / 32;
+    static_assert(WR * WC == kGroup / 32, "warp tiling");
 };
 
 template <int D>
@@ -65,16 +70,24 @@ struct Tile {
         wi = w % FT<D>::WR;
         wj = w / FT<D>::WR;
         i0 = 4 * FT<D>::TI * wi + FT<D>::TI * li;
-        j0 = 32 * wj + 4 * lj;
+        j0 = 8 * FT<D>::TJ * wj + FT<D>::TJ * lj;
     }
 };
 
-// compress scratch: rowE [D] f64 | colE [D] f64 | dred [WC][D] f64 | dredc [WR][D] f64
-// | red [WC][D] | redc [WR][D] | rowv [D] | colv [D] | sm [D] | qs [D] | pick [16] | ctl [16]
+// P[ip][jj] = (S[i0 + 2ip][j0 + jj], S[i0 + 2ip + 1][j0 + jj])
+template <int D>
+using TileReg = float2[FT<D>::IP][FT<D>::TJ];
+
+// scratch: dred [WC][D] f64 | dredc [WR][D] f64 | red [WC][D] | redc [WR][D]
+// | line [2][D] | pick [16]; then D*D bytes of unpacked codes (packed formats)
 template <int D>
 __host__ __device__ constexpr uint32_t compress_scratch_bytes() {
-    return align_up(8u * (2u * D + FT<D>::WC * D + FT<D>::WR * D) +
-                        (FT<D>::WC * D + FT<D>::WR * D + 4u * D + 32u) * 4u, 128u);
+    return align_up(8u * (FT<D>::WC + FT<D>::WR) * D + 4u * ((FT<D>::WC + FT<D>::WR + 2u) * D + 16u), 128u);
+}
+
+template <int D, int BITS>
+__host__ __device__ constexpr uint32_t group_smem_bytes() {
+    return compress_scratch_bytes<D>() + (BITS != 8 ? (uint32_t)D * D : 0u);
 }
 
 // One flush stage: the blob prefix through W buffered pairs.
@@ -84,20 +97,18 @@ __host__ __device__ inline uint32_t flush_stage_bytes(const Layout &L, int windo
 
 constexpr int kFlushStages = 2;
 
-template <int D>
-__host__ __device__ constexpr uint32_t flush_fixed_smem() {
-    return 256u + compress_scratch_bytes<D>();
+inline uint32_t group_smem_for(int D, int bits) {
+    if (D == 128) return bits == 8 ? group_smem_bytes<128, 8>() : group_smem_bytes<128, 4>();
+    return bits == 8 ? group_smem_bytes<64, 8>() : group_smem_bytes<64, 4>();
 }
 
 inline uint32_t flush_smem_bytes(int D, int bits, const Layout &L, int window) {
-    const uint32_t fixed = D == 128 ? flush_fixed_smem<128>() : flush_fixed_smem<64>();
-    return fixed + (bits != 8 ? (uint32_t)D * D : 0u) + kFlushStages * flush_stage_bytes(L, window);
+    return 256u + group_smem_for(D, bits) + kFlushStages * flush_stage_bytes(L, window);
 }
 
 // init / dequant: one blob per CTA
 inline uint32_t boundary_smem_bytes(int D, int bits, const Layout &L, int window) {
-    const uint32_t fixed = D == 128 ? flush_fixed_smem<128>() : flush_fixed_smem<64>();
-    return fixed + (bits != 8 ? (uint32_t)D * D : 0u) + flush_stage_bytes(L, window);
+    return 256u + group_smem_for(D, bits) + flush_stage_bytes(L, window);
 }
 
 struct FlushArgs {
@@ -109,17 +120,18 @@ struct FlushArgs {
     int num_heads;
 };
 
-__device__ __forceinline__ void cons_sync(int n) { asm volatile("bar.sync 2, %0;" ::"r"(n) : "memory"); }
+// barrier of the 256 threads that handle a blob
+__device__ __forceinline__ void gsync() { asm volatile("bar.sync 2, 256;" ::: "memory"); }
 
-__device__ __forceinline__ bool cons_sync_and(bool pred, int n) {
+__device__ __forceinline__ bool gsync_and(bool pred) {
     uint32_t r;
     asm volatile(
         "{\n\t.reg .pred p, q;\n\t"
         "setp.ne.u32 p, %1, 0;\n\t"
-        "bar.red.and.pred q, 2, %2, p;\n\t"
+        "bar.red.and.pred q, 2, 256, p;\n\t"
         "selp.u32 %0, 1, 0, q;\n\t}"
         : "=r"(r)
-        : "r"((uint32_t)pred), "r"(n)
+        : "r"((uint32_t)pred)
         : "memory");
     return r != 0;
 }
@@ -129,9 +141,9 @@ __device__ __forceinline__ float2 f2(float a, float b) { return make_float2(a, b
 template <typename T, bool MAX>
 __device__ __forceinline__ T rop(T a, T b) { return MAX ? (a > b ? a : b) : a + b; }
 
-// Sum (or max) of per-thread row partials r[ii] over the 8 lanes sharing li
-// (lane bits 2..4): reduce-scatter, then lane lj holds the total of row
-// ii = lj * TI / 8 (TI = 8: every lj; TI = 4: lj = 2*ii and 2*ii + 1 both hold it).
+// Row partials r[TI] combined over the 8 lanes sharing li (lane bits 2..4) by
+// reduce-scatter: lane lj ends with row lj * TI / 8 of the thread's tile
+// (TI = 4: lanes 2k and 2k + 1 both hold row k).
 template <int TI, typename T, bool MAX>
 __device__ __forceinline__ T warp_rows(const T (&r)[TI], int lane) {
     T v[TI];
@@ -143,13 +155,12 @@ __device__ __forceinline__ T warp_rows(const T (&r)[TI], int lane) {
         if (n > 1) {
             const bool up = lane & off;
 #pragma unroll
-            for (int i = 0; i < TI / 2; ++i) {
+            for (int i = 0; i < TI / 2; ++i)
                 if (i < n / 2) {
                     const T send = up ? v[i] : v[i + n / 2];
                     const T keep = up ? v[i + n / 2] : v[i];
                     v[i] = rop<T, MAX>(keep, __shfl_xor_sync(0xFFFFFFFFu, send, off));
                 }
-            }
             n >>= 1;
         } else {
             v[0] = rop<T, MAX>(v[0], __shfl_xor_sync(0xFFFFFFFFu, v[0], off));
@@ -158,81 +169,67 @@ __device__ __forceinline__ T warp_rows(const T (&r)[TI], int lane) {
     return v[0];
 }
 
-// Sum (or max) of per-thread column partials c[jj] over the 4 lanes sharing
-// lj (lane bits 0..1): lane li holds the total of column jj = li.
-template <typename T, bool MAX>
-__device__ __forceinline__ T warp_cols(const T (&c)[4], int lane) {
-    T v[4] = {c[0], c[1], c[2], c[3]};
-    {
-        const bool up = lane & 2;
+// Column partials c[TJ] combined over the 4 lanes sharing lj (lane bits
+// 0..1): lane li ends with columns (TJ/4)*li + q, q < TJ/4, in out[q].
+template <int TJ, typename T, bool MAX>
+__device__ __forceinline__ void warp_cols(const T (&c)[TJ], T (&out)[TJ / 4], int lane) {
+    T v[TJ];
 #pragma unroll
-        for (int i = 0; i < 2; ++i) {
-            const T send = up ? v[i] : v[i + 2];
-            const T keep = up ? v[i + 2] : v[i];
-            v[i] = rop<T, MAX>(keep, __shfl_xor_sync(0xFFFFFFFFu, send, 2));
-        }
+    for (int i = 0; i < TJ; ++i) v[i] = c[i];
+    int n = TJ;
+#pragma unroll
+    for (int off = 2; off >= 1; off >>= 1) {
+        const bool up = lane & off;
+#pragma unroll
+        for (int i = 0; i < TJ / 2; ++i)
+            if (i < n / 2) {
+                const T send = up ? v[i] : v[i + n / 2];
+                const T keep = up ? v[i + n / 2] : v[i];
+                v[i] = rop<T, MAX>(keep, __shfl_xor_sync(0xFFFFFFFFu, send, off));
+            }
+        n >>= 1;
     }
-    const bool up = lane & 1;
-    const T send = up ? v[0] : v[1];
-    const T keep = up ? v[1] : v[0];
-    return rop<T, MAX>(keep, __shfl_xor_sync(0xFFFFFFFFu, send, 1));
+#pragma unroll
+    for (int q = 0; q < TJ / 4; ++q) out[q] = v[q];
 }
 
-// Row totals (over j) into rowv and column totals (over i) into colv for
-// float partials; two consumer barriers.
-template <int D, bool MAX>
-__device__ __forceinline__ void reduce_rows_cols(const float (&r)[FT<D>::TI], const float (&c)[4],
-                                                 float *red, float *redc, float *rowv, float *colv,
-                                                 int tid, bool rows, bool cols) {
-    constexpr int TI = FT<D>::TI, NT = FT<D>::NT, WR = FT<D>::WR, WC = FT<D>::WC;
+// Per-warp row partials into red[wj][i], column partials into redc[wi][j].
+template <int D, typename T, bool MAX>
+__device__ __forceinline__ void store_row_partials(const T (&r)[FT<D>::TI], T *red, int tid) {
+    constexpr int TI = FT<D>::TI;
     const Tile<D> t(tid);
-    const int lane = tid & 31;
-    if (rows) {
-        const float v = warp_rows<TI, float, MAX>(r, lane);
-        if (TI == 8 || (t.lj & 1) == 0) red[t.wj * D + t.i0 + t.lj * TI / 8] = v;
-    }
-    if (cols) {
-        const float v = warp_cols<float, MAX>(c, lane);
-        redc[t.wi * D + t.j0 + t.li] = v;
-    }
-    cons_sync(NT);
-    if (rows && tid < D) {
-        float a = red[tid];
+    const T v = warp_rows<TI, T, MAX>(r, tid & 31);
+    if (TI == 8 || (t.lj & 1) == 0) red[t.wj * D + t.i0 + t.lj * TI / 8] = v;
+}
+
+template <int D, typename T, bool MAX>
+__device__ __forceinline__ void store_col_partials(const T (&c)[FT<D>::TJ], T *redc, int tid) {
+    constexpr int TJ = FT<D>::TJ;
+    const Tile<D> t(tid);
+    T o[TJ / 4];
+    warp_cols<TJ, T, MAX>(c, o, tid & 31);
 #pragma unroll
-        for (int w = 1; w < WC; ++w) a = rop<float, MAX>(a, red[w * D + tid]);
-        rowv[tid] = a;
-    }
-    if (cols && tid >= D && tid < 2 * D) {
-        const int j = tid - D;
-        float a = redc[j];
-#pragma unroll
-        for (int w = 1; w < WR; ++w) a = rop<float, MAX>(a, redc[w * D + j]);
-        colv[j] = a;
-    }
-    cons_sync(NT);
+    for (int q = 0; q < TJ / 4; ++q) redc[t.wi * D + t.j0 + (TJ / 4) * t.li + q] = o[q];
 }
 
 // The FP32 state of a blob, in the rule's order (see the file comment).
 // codes8: rows of D signed 8-bit codes (value-major).
 template <int D>
-__device__ __forceinline__ void reconstruct_tile(float (&R)[FT<D>::TI][4], const uint8_t *qs_p,
-                                                 const uint8_t *sm_p, const float *cvec,
-                                                 const int8_t *codes8, const float *pairs,
-                                                 const float *gvec, float gsc, const uint32_t *meta,
-                                                 int ncomp, int count, int f16, int tid) {
-    constexpr int TI = FT<D>::TI;
+__device__ __forceinline__ void reconstruct_tile(TileReg<D> &P, const uint8_t *qs_p, const uint8_t *sm_p,
+                                                 const float *cvec, const int8_t *codes8,
+                                                 const float *pairs, const float *gvec, float gsc,
+                                                 const uint32_t *meta, int ncomp, int count, int f16,
+                                                 int tid) {
+    constexpr int TI = FT<D>::TI, TJ = FT<D>::TJ, IP = FT<D>::IP;
     const Tile<D> t(tid);
     const int i0 = t.i0, j0 = t.j0;
-    float qsj[4], smi[TI], gi[TI];
+    float2 sm2[IP];
 #pragma unroll
-    for (int jj = 0; jj < 4; ++jj) qsj[jj] = load_scale(qs_p, j0 + jj, f16);
+    for (int ip = 0; ip < IP; ++ip)
+        sm2[ip] = f2(load_scale(sm_p, i0 + 2 * ip, f16), load_scale(sm_p, i0 + 2 * ip + 1, f16));
 #pragma unroll
-    for (int ii = 0; ii < TI; ++ii) {
-        smi[ii] = load_scale(sm_p, i0 + ii, f16);
-        gi[ii] = gvec ? gvec[i0 + ii] : gsc;
-    }
-#pragma unroll
-    for (int jj = 0; jj < 4; ++jj) {
+    for (int jj = 0; jj < TJ; ++jj) {
+        const float q = load_scale(qs_p, j0 + jj, f16);
         const int8_t *row = codes8 + (size_t)(j0 + jj) * D + i0;
         uint32_t w[TI / 4];
         if constexpr (TI == 8) {
@@ -243,13 +240,11 @@ __device__ __forceinline__ void reconstruct_tile(float (&R)[FT<D>::TI][4], const
             w[0] = *reinterpret_cast<const uint32_t *>(row) ^ 0x80808080u;
         }
 #pragma unroll
-        for (int ii = 0; ii < TI; ii += 2) {
+        for (int ip = 0; ip < IP; ++ip) {
+            const int ii = 2 * ip;
             float2 cf = f2(byte_to_float(w[ii >> 2], ii & 3), byte_to_float(w[ii >> 2], (ii & 3) + 1));
             cf = __fadd2_rn(cf, f2(-8388736.0f, -8388736.0f));  // exact codes
-            float2 b = __fmul2_rn(cf, f2(qsj[jj], qsj[jj]));
-            b = __fmul2_rn(b, f2(smi[ii], smi[ii + 1]));
-            R[ii][jj] = b.x;
-            R[ii + 1][jj] = b.y;
+            P[ip][jj] = __fmul2_rn(__fmul2_rn(cf, f2(q, q)), sm2[ip]);
         }
     }
     for (int cc = 0; cc < ncomp; ++cc) {
@@ -257,50 +252,57 @@ __device__ __forceinline__ void reconstruct_tile(float (&R)[FT<D>::TI][4], const
         const float *w = cvec + (size_t)cc * D;
         const int idx = (int)(m & 0x7FFFFFFFu);
         if (m & kCompCol) {
-            if (idx >= j0 && idx < j0 + 4) {
+            if (idx >= j0 && idx < j0 + TJ) {
 #pragma unroll
-                for (int jj = 0; jj < 4; ++jj)
+                for (int jj = 0; jj < TJ; ++jj)
                     if (j0 + jj == idx)
 #pragma unroll
-                        for (int ii = 0; ii < TI; ++ii) R[ii][jj] = __fadd_rn(R[ii][jj], w[i0 + ii]);
+                        for (int ip = 0; ip < IP; ++ip)
+                            P[ip][jj] = __fadd2_rn(P[ip][jj], f2(w[i0 + 2 * ip], w[i0 + 2 * ip + 1]));
             }
         } else if (idx >= i0 && idx < i0 + TI) {
 #pragma unroll
-            for (int ii = 0; ii < TI; ++ii)
-                if (i0 + ii == idx)
+            for (int ip = 0; ip < IP; ++ip) {
+                if (i0 + 2 * ip == idx)
 #pragma unroll
-                    for (int jj = 0; jj < 4; ++jj) R[ii][jj] = __fadd_rn(R[ii][jj], w[j0 + jj]);
+                    for (int jj = 0; jj < TJ; ++jj) P[ip][jj].x = __fadd_rn(P[ip][jj].x, w[j0 + jj]);
+                if (i0 + 2 * ip + 1 == idx)
+#pragma unroll
+                    for (int jj = 0; jj < TJ; ++jj) P[ip][jj].y = __fadd_rn(P[ip][jj].y, w[j0 + jj]);
+            }
         }
     }
     for (int m = 0; m < count; ++m) {
         const float *p = pairs + (size_t)m * 2 * D;
-        float kh[TI];
+        float2 kh[IP];
 #pragma unroll
-        for (int ii = 0; ii < TI; ii += 4) {
-            const float4 k4 = *reinterpret_cast<const float4 *>(p + i0 + ii);
-            kh[ii] = k4.x; kh[ii + 1] = k4.y; kh[ii + 2] = k4.z; kh[ii + 3] = k4.w;
+        for (int ip = 0; ip < IP; ip += 2) {
+            const float4 k4 = *reinterpret_cast<const float4 *>(p + i0 + 2 * ip);
+            kh[ip] = f2(k4.x, k4.y);
+            kh[ip + 1] = f2(k4.z, k4.w);
         }
-        const float4 u4 = *reinterpret_cast<const float4 *>(p + D + j0);
-        const float uu[4] = {u4.x, u4.y, u4.z, u4.w};
+        float uu[TJ];
 #pragma unroll
-        for (int ii = 0; ii < TI; ii += 2) {
+        for (int jj = 0; jj < TJ; jj += 4) {
+            const float4 u4 = *reinterpret_cast<const float4 *>(p + D + j0 + jj);
+            uu[jj] = u4.x;
+            uu[jj + 1] = u4.y;
+            uu[jj + 2] = u4.z;
+            uu[jj + 3] = u4.w;
+        }
 #pragma unroll
-            for (int jj = 0; jj < 4; ++jj) {
-                const float2 r = __ffma2_rn(f2(kh[ii], kh[ii + 1]), f2(uu[jj], uu[jj]),
-                                            f2(R[ii][jj], R[ii + 1][jj]));
-                R[ii][jj] = r.x;
-                R[ii + 1][jj] = r.y;
-            }
+        for (int jj = 0; jj < TJ; ++jj) {
+            const float2 u2 = f2(uu[jj], uu[jj]);
+#pragma unroll
+            for (int ip = 0; ip < IP; ++ip) P[ip][jj] = __ffma2_rn(kh[ip], u2, P[ip][jj]);
         }
     }
 #pragma unroll
-    for (int ii = 0; ii < TI; ii += 2)
+    for (int ip = 0; ip < IP; ++ip) {
+        const float2 g2 = gvec ? f2(gvec[i0 + 2 * ip], gvec[i0 + 2 * ip + 1]) : f2(gsc, gsc);
 #pragma unroll
-        for (int jj = 0; jj < 4; ++jj) {
-            const float2 r = __fmul2_rn(f2(gi[ii], gi[ii + 1]), f2(R[ii][jj], R[ii + 1][jj]));
-            R[ii][jj] = r.x;
-            R[ii + 1][jj] = r.y;
-        }
+        for (int jj = 0; jj < TJ; ++jj) P[ip][jj] = __fmul2_rn(g2, P[ip][jj]);
+    }
 }
 
 // smallest power of two >= m (m > 0 finite), clamped to [lo, hi]
@@ -324,238 +326,284 @@ __device__ __forceinline__ float pow2_recip(float s) {
     return e <= 253u ? __uint_as_float((254u - e) << 23) : 0x1p-127f;
 }
 
-// Compress the register tile R (rules in the file comment) and write the new
+// the low bytes of four words, in order
+__device__ __forceinline__ uint32_t pack4_low_bytes(uint32_t a, uint32_t b, uint32_t c, uint32_t d) {
+    return __byte_perm(__byte_perm(a, b, 0x0040), __byte_perm(c, d, 0x0040), 0x5410);
+}
+
+// Compress the register tile P (rules in the file comment) and write the new
 // compact state into `blob`: compensator lines, smoothing and quantization
-// scales, codes, compensator meta.  `scratch` is compress_scratch_bytes<D>()
-// of shared memory; codes8 (packed formats only) D*D bytes.  Returns the
-// number of compensators taken.  Every consumer thread must call it.
+// scales, codes, compensator meta.  `scratch` is group_smem_bytes<D, BITS>()
+// of shared memory.  Returns the number of compensators taken.  All 256
+// consumers must call it.
 template <int D, int BITS>
-__device__ int compress_tile(float (&R)[FT<D>::TI][4], const Flags &F, const Layout &L,
-                             uint8_t *scratch, int8_t *codes8, uint8_t *blob, int tid) {
-    constexpr int TI = FT<D>::TI, NT = FT<D>::NT, WR = FT<D>::WR, WC = FT<D>::WC;
-    constexpr int QMAX = (1 << (BITS - 1)) - 1;
+__device__ int compress_tile(TileReg<D> &P, const Flags &F, const Layout &L, uint8_t *scratch,
+                             uint8_t *blob, int tid) {
+    constexpr int TI = FT<D>::TI, TJ = FT<D>::TJ, IP = FT<D>::IP, WR = FT<D>::WR, WC = FT<D>::WC;
+    constexpr int KE = FT<D>::KE, QMAX = (1 << (BITS - 1)) - 1;
     const Tile<D> t(tid);
     const int lane = tid & 31, i0 = t.i0, j0 = t.j0;
-    double *rowE = reinterpret_cast<double *>(scratch);
-    double *colE = rowE + D;
-    double *dred = colE + D;         // [WC][D]
-    double *dredc = dred + WC * D;   // [WR][D]
+    double *dred = reinterpret_cast<double *>(scratch);  // [WC][D]
+    double *dredc = dred + WC * D;                        // [WR][D]
     float *red = reinterpret_cast<float *>(dredc + WR * D);
     float *redc = red + WC * D;
-    float *rowv = redc + WR * D, *colv = rowv + D, *smv = colv + D, *qsv = smv + D;
-    uint32_t *pick = reinterpret_cast<uint32_t *>(qsv + D);
+    float *line = redc + WR * D;  // [2][D]
+    uint32_t *pick = reinterpret_cast<uint32_t *>(line + 2 * D);
+    int8_t *codes8 = reinterpret_cast<int8_t *>(scratch + compress_scratch_bytes<D>());
     float *cvec_out = reinterpret_cast<float *>(blob + L.cvec_off);
 
-    // ---- line energies in FP64 (exact squares), then greedy one-hot extraction;
-    // taking a line only lowers the other side's energies, updated in place
+    // ---- line energies (FP64 sums of exact squares); lane l of every warp
+    // keeps rows and columns l + 32k
+    double rE[KE], cE[KE];
     if (F.num_comp > 0) {
-        double er[TI], ec[4] = {0.0, 0.0, 0.0, 0.0};
-#pragma unroll
-        for (int ii = 0; ii < TI; ++ii) {
-            er[ii] = 0.0;
-#pragma unroll
-            for (int jj = 0; jj < 4; ++jj) {
-                const double x = (double)R[ii][jj];
-                er[ii] = fma(x, x, er[ii]);
-                ec[jj] = fma(x, x, ec[jj]);
-            }
-        }
         {
-            const double v = warp_rows<TI, double, false>(er, lane);
-            if (TI == 8 || (t.lj & 1) == 0) dred[t.wj * D + i0 + t.lj * TI / 8] = v;
-            const double w = warp_cols<double, false>(ec, lane);
-            dredc[t.wi * D + j0 + t.li] = w;
-        }
-        cons_sync(NT);
-        if (tid < D) {
-            double a = dred[tid];
+            double er[TI], ec[TJ];
 #pragma unroll
-            for (int w = 1; w < WC; ++w) a += dred[w * D + tid];
-            rowE[tid] = a;
-        } else if (tid < 2 * D) {
-            const int j = tid - D;
-            double a = dredc[j];
+            for (int i = 0; i < TI; ++i) er[i] = 0.0;
 #pragma unroll
-            for (int w = 1; w < WR; ++w) a += dredc[w * D + j];
-            colE[j] = a;
+            for (int j = 0; j < TJ; ++j) ec[j] = 0.0;
+#pragma unroll
+            for (int ip = 0; ip < IP; ++ip)
+#pragma unroll
+                for (int jj = 0; jj < TJ; ++jj) {
+                    const double a = (double)P[ip][jj].x, b = (double)P[ip][jj].y;
+                    er[2 * ip] = fma(a, a, er[2 * ip]);
+                    er[2 * ip + 1] = fma(b, b, er[2 * ip + 1]);
+                    ec[jj] = fma(b, b, fma(a, a, ec[jj]));
+                }
+            store_row_partials<D, double, false>(er, dred, tid);
+            store_col_partials<D, double, false>(ec, dredc, tid);
         }
-        cons_sync(NT);
+        gsync();
+#pragma unroll
+        for (int k = 0; k < KE; ++k) {
+            const int x = lane + 32 * k;
+            double a = dred[x], b = dredc[x];
+#pragma unroll
+            for (int w = 1; w < WC; ++w) a += dred[w * D + x];
+#pragma unroll
+            for (int w = 1; w < WR; ++w) b += dredc[w * D + x];
+            rE[k] = a;
+            cE[k] = b;
+        }
     }
+
+    // ---- greedy one-hot extraction, one barrier per round
     int ncomp = 0;
     for (int cc = 0; cc < F.num_comp; ++cc) {
-        if (tid < 32) {
-            double best = -1.0;
-            int key = 0x7FFFFFFF;
+        // Non-negative doubles order like their bit patterns (negative
+        // rounding residue never wins against 0).  Keys: rows 0..D-1, then
+        // columns D..2D-1; strict comparisons in key order keep the lower key.
+        long long bb = 0;
+        uint32_t key = 0xFFFFFFFFu;
 #pragma unroll
-            for (int x = 0; x < 2 * D / 32; ++x) {
-                const int k = lane + 32 * x;
-                const double e = k < D ? rowE[k] : colE[k - D];
-                if (e > best) { best = e; key = k; }  // ascending keys: ties keep the lower key
-            }
-#pragma unroll
-            for (int off = 16; off >= 1; off >>= 1) {
-                const double ob = __shfl_xor_sync(0xFFFFFFFFu, best, off);
-                const int ok = __shfl_xor_sync(0xFFFFFFFFu, key, off);
-                if (ob > best || (ob == best && ok < key)) { best = ob; key = ok; }
-            }
-            if (lane == 0) {
-                uint32_t p = kCompNone;
-                if (best > 0.0) {
-                    p = key < D ? (uint32_t)key : (kCompCol | (uint32_t)(key - D));
-                    if (key < D) rowE[key] = 0.0; else colE[key - D] = 0.0;
-                }
-                pick[cc] = p;
-            }
+        for (int k = 0; k < KE; ++k) {
+            const long long e = __double_as_longlong(rE[k]);
+            if (e > bb) { bb = e; key = lane + 32 * k; }
         }
-        cons_sync(NT);
-        const uint32_t p = pick[cc];
-        if (p == kCompNone) break;
-        float *w = cvec_out + (size_t)cc * D;
-        const int idx = (int)(p & 0x7FFFFFFFu);
-        if (p & kCompCol) {
-            if (idx >= j0 && idx < j0 + 4) {
 #pragma unroll
-                for (int jj = 0; jj < 4; ++jj)
+        for (int k = 0; k < KE; ++k) {
+            const long long e = __double_as_longlong(cE[k]);
+            if (e > bb) { bb = e; key = D + lane + 32 * k; }
+        }
+        const uint32_t hi = (uint32_t)((unsigned long long)bb >> 32), lo = (uint32_t)bb;
+        const uint32_t mhi = __reduce_max_sync(0xFFFFFFFFu, hi);
+        const uint32_t mlo = __reduce_max_sync(0xFFFFFFFFu, hi == mhi ? lo : 0u);
+        if ((mhi | mlo) == 0u) break;  // no energy left: the same in every warp
+        key = __reduce_min_sync(0xFFFFFFFFu, (hi == mhi && lo == mlo) ? key : 0xFFFFFFFFu);
+        const bool col = key >= (uint32_t)D;
+        const int idx = col ? (int)key - D : (int)key;
+        if (tid == 0) pick[cc] = col ? (kCompCol | (uint32_t)idx) : (uint32_t)idx;
+        float *w = cvec_out + (size_t)cc * D;
+        float *ln = line + (cc & 1) * D;
+        if (col) {
+            if (idx >= j0 && idx < j0 + TJ) {
+#pragma unroll
+                for (int jj = 0; jj < TJ; ++jj)
                     if (j0 + jj == idx) {
 #pragma unroll
-                        for (int ii = 0; ii < TI; ++ii) {
-                            const float x = R[ii][jj];
-                            w[i0 + ii] = x;
-                            rowE[i0 + ii] -= (double)x * (double)x;
-                            R[ii][jj] = 0.f;
+                        for (int ip = 0; ip < IP; ip += 2) {
+                            const float4 v = make_float4(P[ip][jj].x, P[ip][jj].y, P[ip + 1][jj].x, P[ip + 1][jj].y);
+                            *reinterpret_cast<float4 *>(w + i0 + 2 * ip) = v;
+                            *reinterpret_cast<float4 *>(ln + i0 + 2 * ip) = v;
+                            P[ip][jj] = f2(0.f, 0.f);
+                            P[ip + 1][jj] = f2(0.f, 0.f);
                         }
                     }
             }
         } else if (idx >= i0 && idx < i0 + TI) {
 #pragma unroll
-            for (int ii = 0; ii < TI; ++ii)
-                if (i0 + ii == idx) {
-                    *reinterpret_cast<float4 *>(w + j0) = make_float4(R[ii][0], R[ii][1], R[ii][2], R[ii][3]);
+            for (int ip = 0; ip < IP; ++ip) {
+                if (i0 + 2 * ip == idx) {
 #pragma unroll
-                    for (int jj = 0; jj < 4; ++jj) {
-                        colE[j0 + jj] -= (double)R[ii][jj] * (double)R[ii][jj];
-                        R[ii][jj] = 0.f;
+                    for (int jj = 0; jj < TJ; jj += 4) {
+                        const float4 v = make_float4(P[ip][jj].x, P[ip][jj + 1].x, P[ip][jj + 2].x, P[ip][jj + 3].x);
+                        *reinterpret_cast<float4 *>(w + j0 + jj) = v;
+                        *reinterpret_cast<float4 *>(ln + j0 + jj) = v;
                     }
+#pragma unroll
+                    for (int jj = 0; jj < TJ; ++jj) P[ip][jj].x = 0.f;
                 }
+                if (i0 + 2 * ip + 1 == idx) {
+#pragma unroll
+                    for (int jj = 0; jj < TJ; jj += 4) {
+                        const float4 v = make_float4(P[ip][jj].y, P[ip][jj + 1].y, P[ip][jj + 2].y, P[ip][jj + 3].y);
+                        *reinterpret_cast<float4 *>(w + j0 + jj) = v;
+                        *reinterpret_cast<float4 *>(ln + j0 + jj) = v;
+                    }
+#pragma unroll
+                    for (int jj = 0; jj < TJ; ++jj) P[ip][jj].y = 0.f;
+                }
+            }
+        }
+        gsync();
+        // taking a row lowers every column's energy by the row entry's square
+        // (and the reverse); the taken line drops out
+#pragma unroll
+        for (int k = 0; k < KE; ++k) {
+            const int x = lane + 32 * k;
+            const double v = (double)ln[x];
+            if (col) {
+                rE[k] -= v * v;
+                if (x == idx) cE[k] = 0.0;
+            } else {
+                cE[k] -= v * v;
+                if (x == idx) rE[k] = 0.0;
+            }
         }
         ++ncomp;
-        cons_sync(NT);
     }
     for (int cc = ncomp; cc < F.num_comp; ++cc)
-        for (int x = tid; x < D; x += NT) cvec_out[(size_t)cc * D + x] = 0.f;
+        for (int x = tid; x < D; x += kGroup) cvec_out[(size_t)cc * D + x] = 0.f;
 
     // ---- residual smoothing: one power of two per key row
     const float sm_lo = F.f16_scale ? 0x1p-14f : 0x1p-126f;
     const float sm_hi = F.f16_scale ? 0x1p15f : 0x1p127f;
     {
-        float mr[TI], dummy[4] = {0.f, 0.f, 0.f, 0.f};
+        float mr[TI];
 #pragma unroll
-        for (int ii = 0; ii < TI; ++ii)
-            mr[ii] = fmaxf(fmaxf(fabsf(R[ii][0]), fabsf(R[ii][1])), fmaxf(fabsf(R[ii][2]), fabsf(R[ii][3])));
-        reduce_rows_cols<D, true>(mr, dummy, red, redc, rowv, colv, tid, true, false);
-        if (tid < D) {
-            const float m = rowv[tid];
-            const float s = (F.smoothing && m > 0.f) ? pow2_ceil_clamped(m, sm_lo, sm_hi) : 1.f;
-            smv[tid] = s;
-            if (F.f16_scale) reinterpret_cast<__half *>(blob + L.sm_off)[tid] = __float2half_rn(s);
-            else reinterpret_cast<float *>(blob + L.sm_off)[tid] = s;
+        for (int ip = 0; ip < IP; ++ip) {
+            float a = 0.f, b = 0.f;
+#pragma unroll
+            for (int jj = 0; jj < TJ; ++jj) {
+                a = fmaxf(a, fabsf(P[ip][jj].x));
+                b = fmaxf(b, fabsf(P[ip][jj].y));
+            }
+            mr[2 * ip] = a;
+            mr[2 * ip + 1] = b;
         }
-        cons_sync(NT);
+        store_row_partials<D, float, true>(mr, red, tid);
     }
-    float cm[4] = {0.f, 0.f, 0.f, 0.f};
+    gsync();
+    float cm[TJ];
 #pragma unroll
-    for (int ii = 0; ii < TI; ii += 2) {
-        const float2 inv = f2(pow2_recip(smv[i0 + ii]), pow2_recip(smv[i0 + ii + 1]));
+    for (int jj = 0; jj < TJ; ++jj) cm[jj] = 0.f;
+    {
+        // lane lj finishes row i0 + lj*TI/8 (the row warp_rows left it), then
+        // the 8 lanes sharing li swap their scales
+        const int r = i0 + t.lj * TI / 8;
+        float m = red[r];
 #pragma unroll
-        for (int jj = 0; jj < 4; ++jj) {
-            const float2 r = __fmul2_rn(f2(R[ii][jj], R[ii + 1][jj]), inv);  // exact
-            R[ii][jj] = r.x;
-            R[ii + 1][jj] = r.y;
-            cm[jj] = fmaxf(cm[jj], fmaxf(fabsf(r.x), fabsf(r.y)));
+        for (int w = 1; w < WC; ++w) m = fmaxf(m, red[w * D + r]);
+        const float sr = (F.smoothing && m > 0.f) ? pow2_ceil_clamped(m, sm_lo, sm_hi) : 1.f;
+        if (t.wj == 0 && (TI == 8 || (t.lj & 1) == 0)) {
+            if (F.f16_scale) reinterpret_cast<__half *>(blob + L.sm_off)[r] = __float2half_rn(sr);
+            else reinterpret_cast<float *>(blob + L.sm_off)[r] = sr;
+        }
+        float smr[TI];
+#pragma unroll
+        for (int ii = 0; ii < TI; ++ii) smr[ii] = __shfl_sync(0xFFFFFFFFu, sr, (ii * 8 / TI) * 4 + t.li);
+#pragma unroll
+        for (int ip = 0; ip < IP; ++ip) {
+            const float2 inv = f2(pow2_recip(smr[2 * ip]), pow2_recip(smr[2 * ip + 1]));
+#pragma unroll
+            for (int jj = 0; jj < TJ; ++jj) {
+                P[ip][jj] = __fmul2_rn(P[ip][jj], inv);  // exact
+                cm[jj] = fmaxf(cm[jj], fmaxf(fabsf(P[ip][jj].x), fabsf(P[ip][jj].y)));
+            }
         }
     }
 
     // ---- symmetric scale per value column
-    {
-        float dummy[TI];
+    store_col_partials<D, float, true>(cm, redc, tid);
+    gsync();
+    // lane li finishes columns j0 + (TJ/4)*li + q (those warp_cols left
+    // it), then the 4 lanes sharing lj swap their scales
+    constexpr int CQ = TJ / 4;
+    float sq[CQ];
 #pragma unroll
-        for (int ii = 0; ii < TI; ++ii) dummy[ii] = 0.f;
-        reduce_rows_cols<D, true>(dummy, cm, red, redc, rowv, colv, tid, false, true);
-    }
-    if (tid < D) {
-        const float m = colv[tid];
+    for (int q = 0; q < CQ; ++q) {
+        const int j = j0 + CQ * t.li + q;
+        float m = redc[j];
+#pragma unroll
+        for (int w = 1; w < WR; ++w) m = fmaxf(m, redc[w * D + j]);
         float s = __fdiv_rn(m, (float)QMAX);
         if (F.f16_scale) {
             s = __half2float(__float2half_rn(s));
             if (m > 0.f && s == 0.f) s = 0x1p-24f;
-            reinterpret_cast<__half *>(blob + L.qs_off)[tid] = __float2half_rn(s);
-        } else {
-            if (m > 0.f && s == 0.f) s = 0x1p-149f;
-            reinterpret_cast<float *>(blob + L.qs_off)[tid] = s;
+        } else if (m > 0.f && s == 0.f) {
+            s = 0x1p-149f;
         }
-        qsv[tid] = s;
+        sq[q] = s;
+        if (t.wi == 0) {
+            if (F.f16_scale) reinterpret_cast<__half *>(blob + L.qs_off)[j] = __float2half_rn(s);
+            else reinterpret_cast<float *>(blob + L.qs_off)[j] = s;
+        }
     }
-    cons_sync(NT);
+    float qsj[TJ];
+#pragma unroll
+    for (int jj = 0; jj < TJ; ++jj) qsj[jj] = __shfl_sync(0xFFFFFFFFu, sq[jj % CQ], (lane & ~3) | (jj / CQ));
 
     // ---- codes: rint of the correctly rounded FP32 quotient, ties to even.
     // Fast path: multiply by the rounded reciprocal (within 1.5 ulp of the
-    // quotient) and round by adding 1.5*2^23.  A thread with any entry within
-    // 2e-5 of a half-integer, or with a column scale so small that the
-    // quotient may leave [-Qmax, Qmax], redoes its entries by division.
+    // quotient) and round by adding 1.5*2^23.  A column with an entry within
+    // 2e-5 of a half-integer, or with a scale so small that the quotient may
+    // leave [-Qmax, Qmax], is redone by division.
     int8_t *dst8 = BITS == 8 ? reinterpret_cast<int8_t *>(blob + L.codes_off) : codes8;
     const uint32_t dst_row = BITS == 8 ? L.row_bytes : (uint32_t)D;
     const float min_fast = F.f16_scale ? 0x1p-14f : 0x1p-100f;
-    float sj[4], inv[4];
-    bool slow = false;
 #pragma unroll
-    for (int jj = 0; jj < 4; ++jj) {
-        sj[jj] = qsv[j0 + jj];
-        inv[jj] = __frcp_rn(sj[jj]);
-        slow |= (sj[jj] != 0.f) && !(sj[jj] >= min_fast);
-    }
-    uint32_t nb[TI][4];
-    float dmax = 0.f;
+    for (int jj = 0; jj < TJ; ++jj) {
+        const float s = qsj[jj];
+        const float inv = __frcp_rn(s);
+        uint32_t nb[TI];
+        float dmax = 0.f;
 #pragma unroll
-    for (int jj = 0; jj < 4; ++jj) {
-#pragma unroll
-        for (int ii = 0; ii < TI; ii += 2) {
-            const float2 tq = __fmul2_rn(f2(R[ii][jj], R[ii + 1][jj]), f2(inv[jj], inv[jj]));
+        for (int ip = 0; ip < IP; ++ip) {
+            const float2 tq = __fmul2_rn(P[ip][jj], f2(inv, inv));
             const float2 nf = __fadd2_rn(tq, f2(12582912.0f, 12582912.0f));  // 1.5 * 2^23
             const float2 back = __fadd2_rn(nf, f2(-12582912.0f, -12582912.0f));
             const float2 d = __fadd2_rn(tq, f2(-back.x, -back.y));
             dmax = fmaxf(dmax, fmaxf(fabsf(d.x), fabsf(d.y)));
-            nb[ii][jj] = sj[jj] != 0.f ? __float_as_uint(nf.x) : 0x4B400000u;
-            nb[ii + 1][jj] = sj[jj] != 0.f ? __float_as_uint(nf.y) : 0x4B400000u;
+            nb[2 * ip] = __float_as_uint(nf.x);
+            nb[2 * ip + 1] = __float_as_uint(nf.y);
         }
-    }
-    if (slow || dmax > 0.49998f) {
+        if (s == 0.f) {
 #pragma unroll
-        for (int jj = 0; jj < 4; ++jj)
+            for (int ii = 0; ii < TI; ++ii) nb[ii] = 0u;
+        } else if (!(s >= min_fast) || dmax > 0.49998f) {
 #pragma unroll
-            for (int ii = 0; ii < TI; ++ii) {
-                if (sj[jj] == 0.f) continue;
-                float tq = __fdiv_rn(R[ii][jj], sj[jj]);
-                tq = fminf(fmaxf(tq, -(float)QMAX), (float)QMAX);
-                nb[ii][jj] = __float_as_uint(__fadd_rn(tq, 12582912.0f));
+            for (int ip = 0; ip < IP; ++ip) {
+                float a = __fdiv_rn(P[ip][jj].x, s), b = __fdiv_rn(P[ip][jj].y, s);
+                a = fminf(fmaxf(a, -(float)QMAX), (float)QMAX);
+                b = fminf(fmaxf(b, -(float)QMAX), (float)QMAX);
+                nb[2 * ip] = __float_as_uint(__fadd_rn(a, 12582912.0f));
+                nb[2 * ip + 1] = __float_as_uint(__fadd_rn(b, 12582912.0f));
             }
-    }
-#pragma unroll
-    for (int jj = 0; jj < 4; ++jj) {
+        }
         int8_t *row = dst8 + (size_t)(j0 + jj) * dst_row + i0;
-        const uint32_t w0 = __byte_perm(__byte_perm(nb[0][jj], nb[1][jj], 0x0040),
-                                        __byte_perm(nb[2][jj], nb[3][jj], 0x0040), 0x5410);
+        const uint32_t w0 = pack4_low_bytes(nb[0], nb[1], nb[2], nb[3]);
         if constexpr (TI == 8) {
-            const uint32_t w1 = __byte_perm(__byte_perm(nb[4][jj], nb[5][jj], 0x0040),
-                                            __byte_perm(nb[6][jj], nb[7][jj], 0x0040), 0x5410);
+            const uint32_t w1 = pack4_low_bytes(nb[4], nb[5], nb[6], nb[7]);
             *reinterpret_cast<uint2 *>(row) = make_uint2(w0, w1);
         } else {
             *reinterpret_cast<uint32_t *>(row) = w0;
         }
     }
     if constexpr (BITS != 8) {
-        cons_sync(NT);
+        gsync();
         constexpr int GB = group_bytes<BITS>(), GPR = D / 16;
-        for (int gi = tid; gi < D * GPR; gi += NT) {
+        for (int gi = tid; gi < D * GPR; gi += kGroup) {
             const int j = gi / GPR, grp = gi % GPR;
             const uint4 w = *reinterpret_cast<const uint4 *>(codes8 + (size_t)j * D + 16 * grp);
             const uint32_t ws[4] = {w.x, w.y, w.z, w.w};
@@ -569,7 +617,7 @@ __device__ int compress_tile(float (&R)[FT<D>::TI][4], const Flags &F, const Lay
         const uint32_t m = tid < ncomp ? pick[tid] : kCompNone;
         reinterpret_cast<uint32_t *>(blob + kHdrMeta)[tid] = m;
     }
-    cons_sync(NT);  // scratch free for the next blob
+    gsync();  // scratch free for the next blob
     return ncomp;
 }
 
@@ -577,8 +625,8 @@ __device__ int compress_tile(float (&R)[FT<D>::TI][4], const Flags &F, const Lay
 template <int D, int BITS>
 __device__ __forceinline__ void unpack_all(const uint8_t *codes, uint32_t row_bytes, int8_t *codes8,
                                            int tid) {
-    constexpr int GB = group_bytes<BITS>(), GPR = D / 16, NT = FT<D>::NT;
-    for (int g = tid; g < D * GPR; g += NT) {
+    constexpr int GB = group_bytes<BITS>(), GPR = D / 16;
+    for (int g = tid; g < D * GPR; g += kGroup) {
         const int j = g / GPR, grp = g % GPR;
         float cf[16];
         unpack16<BITS>(codes + (size_t)j * row_bytes + grp * GB, cf);
@@ -615,10 +663,10 @@ template <int D>
 __device__ __forceinline__ void write_fresh_header(uint8_t *blob, const Flags &F, int ncomp,
                                                    bool reset_status, int tid) {
     if (F.kda)
-        for (int x = tid; x < D; x += FT<D>::NT) reinterpret_cast<float *>(blob + kHdrBytes)[x] = 1.f;
+        for (int x = tid; x < D; x += kGroup) reinterpret_cast<float *>(blob + kHdrBytes)[x] = 1.f;
     if (tid == 0) {
         uint32_t *h = reinterpret_cast<uint32_t *>(blob);
-        h[0] = 0u;                  // count
+        h[0] = 0u;  // count
         if (reset_status) h[1] = 0u;
         h[2] = (uint32_t)ncomp;
         h[3] = kMagic;
@@ -627,10 +675,20 @@ __device__ __forceinline__ void write_fresh_header(uint8_t *blob, const Flags &F
 }
 
 // ---------------------------------------------------------------- flush
+// Bytes staged for a blob whose window holds c pairs: the compact state and
+// the pairs, or only the header when there is nothing to flush (or the count
+// is invalid, which the consumers then report).
+__device__ __forceinline__ uint32_t staged_bytes(const Layout &L, int window, uint32_t c) {
+    return (c == 0u || c > (uint32_t)window) ? (uint32_t)kHdrBytes : L.pairs_off + c * L.pair_bytes;
+}
+
+// Persistent: CTA b flushes blobs b, b + G, b + 2G, ... through two stages.
+// Thread 0 stages blob it + 2 as soon as every consumer has rebuilt blob it
+// (the barrier after the rebuild frees the stage); it reads that blob's
+// window count at the top of the iteration, so the load is long done.
 template <int D, int BITS>
-__global__ void __launch_bounds__(4 * D + 32, 1) flush_kernel(FlushArgs A) {
-    constexpr int NT = FT<D>::NT, TI = FT<D>::TI;
-    const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
+__global__ void __launch_bounds__(kGroup, 2) flush_kernel(FlushArgs A) {
+    const int tid = threadIdx.x;
     const Layout L = A.L;
     const Flags F = A.F;
     const uint32_t SB = flush_stage_bytes(L, F.window);
@@ -639,58 +697,36 @@ __global__ void __launch_bounds__(4 * D + 32, 1) flush_kernel(FlushArgs A) {
 
     extern __shared__ __align__(128) uint8_t smem[];
     uint64_t *full = reinterpret_cast<uint64_t *>(smem);
-    uint64_t *empty = full + kFlushStages;
-    volatile uint32_t *s_abort = reinterpret_cast<volatile uint32_t *>(smem + 60);
-    uint32_t *s_cnt = reinterpret_cast<uint32_t *>(smem + 64);  // producer batch [32]
     uint8_t *scratch = smem + 256;
     int8_t *codes8 = reinterpret_cast<int8_t *>(scratch + compress_scratch_bytes<D>());
-    uint8_t *stages = reinterpret_cast<uint8_t *>(codes8) + (BITS != 8 ? D * D : 0);
+    uint8_t *stages = scratch + group_smem_bytes<D, BITS>();
+    auto blob_at = [&](int it) { return A.state + ((size_t)blockIdx.x + (size_t)it * G) * L.blob; };
 
     if (tid == 0) {
-        for (int s = 0; s < kFlushStages; ++s) {
-            mbar_init(&full[s], 1);
-            mbar_init(&empty[s], 1);
-        }
-        *s_abort = 0u;
+        for (int s = 0; s < kFlushStages; ++s) mbar_init(&full[s], 1);
         fence_mbar_init();
+        for (int it = 0; it < kFlushStages && it < n_mine; ++it) {
+            const uint32_t c = *reinterpret_cast<const uint32_t *>(blob_at(it) + kHdrCount);
+            const uint32_t bytes = staged_bytes(L, F.window, c);
+            mbar_arrive_expect_tx(&full[it], bytes);
+            bulk_g2s(stages + (size_t)it * SB, blob_at(it), bytes, &full[it]);
+        }
     }
     __syncthreads();
-
-    if (warp == NT / 32) {
-        // producer: copy each blob's prefix and its buffered pairs; the
-        // window counts of up to 32 blobs are read at once
-        for (int base = 0; base < n_mine && !*s_abort; base += 32) {
-            if (base + lane < n_mine)
-                s_cnt[lane] = *reinterpret_cast<const uint32_t *>(
-                    A.state + ((size_t)blockIdx.x + (size_t)(base + lane) * G) * L.blob + kHdrCount);
-            __syncwarp();
-            if (lane == 0) {
-                for (int x = 0; x < 32 && base + x < n_mine; ++x) {
-                    const int it = base + x, s = it % kFlushStages;
-                    if (it >= kFlushStages && !mbar_wait_bounded(&empty[s], ((it / kFlushStages) - 1) & 1)) {
-                        *s_abort = 1u;
-                        break;
-                    }
-                    const uint8_t *blob = A.state + ((size_t)blockIdx.x + (size_t)it * G) * L.blob;
-                    const uint32_t c = s_cnt[x];
-                    const uint32_t bytes = L.pairs_off + (c <= (uint32_t)F.window ? c : 0u) * L.pair_bytes;
-                    mbar_arrive_expect_tx(&full[s], bytes);
-                    bulk_g2s(stages + (size_t)s * SB, blob, bytes, &full[s]);
-                }
-            }
-            __syncwarp();
-        }
-        return;
-    }
 
     for (int it = 0; it < n_mine; ++it) {
         const int s = it % kFlushStages;
         const uint8_t *st = stages + (size_t)s * SB;
-        uint8_t *blob = A.state + ((size_t)blockIdx.x + (size_t)it * G) * L.blob;
-        if (!cons_sync_and(mbar_wait_bounded(&full[s], (uint32_t)(it / kFlushStages) & 1u), NT)) {
+        uint8_t *blob = blob_at(it);
+        const bool refill = tid == 0 && it + kFlushStages < n_mine;
+        uint32_t c_next = 0;
+        if (refill) c_next = *reinterpret_cast<const volatile uint32_t *>(blob_at(it + kFlushStages) + kHdrCount);
+        if (!gsync_and(mbar_wait_bounded(&full[s], (uint32_t)(it / kFlushStages) & 1u))) {
             if (tid == 0) {
                 set_status(blob, LQ_DEV_TIMEOUT);
-                *s_abort = 1u;
+                // let the copies still in flight land before the CTA leaves
+                for (int x = it; x < it + kFlushStages && x < n_mine; ++x)
+                    mbar_wait_bounded(&full[x % kFlushStages], (uint32_t)(x / kFlushStages) & 1u);
             }
             break;
         }
@@ -698,25 +734,29 @@ __global__ void __launch_bounds__(4 * D + 32, 1) flush_kernel(FlushArgs A) {
         // flush only a valid blob with a non-empty window and no error flag
         const bool run = H.ok && H.status == 0 && H.count > 0;
         if (!H.ok && tid == 0) set_status(blob, LQ_DEV_CORRUPT);
-        float R[TI][4];
+        TileReg<D> P;
         if (run) {
             const int8_t *c8 = reinterpret_cast<const int8_t *>(st + L.codes_off);
             if constexpr (BITS != 8) {
                 unpack_all<D, BITS>(st + L.codes_off, L.row_bytes, codes8, tid);
-                cons_sync(NT);
+                gsync();
                 c8 = codes8;
             }
-            reconstruct_tile<D>(R, st + L.qs_off, st + L.sm_off,
+            reconstruct_tile<D>(P, st + L.qs_off, st + L.sm_off,
                                 reinterpret_cast<const float *>(st + L.cvec_off), c8,
                                 reinterpret_cast<const float *>(st + L.pairs_off),
                                 F.kda ? reinterpret_cast<const float *>(st + L.g_off) : nullptr, H.g,
                                 reinterpret_cast<const uint32_t *>(st + kHdrMeta), (int)H.ncomp,
                                 (int)H.count, F.f16_scale, tid);
         }
-        cons_sync(NT);  // the stage has been read
-        if (tid == 0) mbar_arrive(&empty[s]);
+        gsync();  // the stage has been read
+        if (refill) {
+            const uint32_t bytes = staged_bytes(L, F.window, c_next);
+            mbar_arrive_expect_tx(&full[s], bytes);
+            bulk_g2s(stages + (size_t)s * SB, blob_at(it + kFlushStages), bytes, &full[s]);
+        }
         if (run) {
-            const int ncomp = compress_tile<D, BITS>(R, F, L, scratch, codes8, blob, tid);
+            const int ncomp = compress_tile<D, BITS>(P, F, L, scratch, blob, tid);
             write_fresh_header<D>(blob, F, ncomp, false, tid);
         }
     }
@@ -724,8 +764,8 @@ __global__ void __launch_bounds__(4 * D + 32, 1) flush_kernel(FlushArgs A) {
 
 // ------------------------------------------------- init (MODE 1), dequant (MODE 2)
 template <int D, int BITS, int MODE>
-__global__ void __launch_bounds__(4 * D) boundary_kernel(FlushArgs A) {
-    constexpr int NT = FT<D>::NT, TI = FT<D>::TI;
+__global__ void __launch_bounds__(kGroup) boundary_kernel(FlushArgs A) {
+    constexpr int IP = FT<D>::IP, TJ = FT<D>::TJ;
     const int tid = threadIdx.x;
     const size_t head = blockIdx.x;
     const Layout L = A.L;
@@ -739,17 +779,23 @@ __global__ void __launch_bounds__(4 * D) boundary_kernel(FlushArgs A) {
     uint32_t *s_hdr = reinterpret_cast<uint32_t *>(smem + 16);
     uint8_t *scratch = smem + 256;
     int8_t *codes8 = reinterpret_cast<int8_t *>(scratch + compress_scratch_bytes<D>());
-    uint8_t *st = reinterpret_cast<uint8_t *>(codes8) + (BITS != 8 ? D * D : 0);
+    uint8_t *st = scratch + group_smem_bytes<D, BITS>();
 
-    float R[TI][4];
+    TileReg<D> P;
     if constexpr (MODE == 1) {
         const float *S0 = A.S0 + head * (size_t)D * D;
 #pragma unroll
-        for (int ii = 0; ii < TI; ++ii) {
-            const float4 r4 = *reinterpret_cast<const float4 *>(S0 + (size_t)(i0 + ii) * D + j0);
-            R[ii][0] = r4.x; R[ii][1] = r4.y; R[ii][2] = r4.z; R[ii][3] = r4.w;
-        }
-        const int ncomp = compress_tile<D, BITS>(R, F, L, scratch, codes8, blob, tid);
+        for (int ip = 0; ip < IP; ++ip)
+#pragma unroll
+            for (int jj = 0; jj < TJ; jj += 4) {
+                const float4 a = *reinterpret_cast<const float4 *>(S0 + (size_t)(i0 + 2 * ip) * D + j0 + jj);
+                const float4 b = *reinterpret_cast<const float4 *>(S0 + (size_t)(i0 + 2 * ip + 1) * D + j0 + jj);
+                P[ip][jj] = f2(a.x, b.x);
+                P[ip][jj + 1] = f2(a.y, b.y);
+                P[ip][jj + 2] = f2(a.z, b.z);
+                P[ip][jj + 3] = f2(a.w, b.w);
+            }
+        const int ncomp = compress_tile<D, BITS>(P, F, L, scratch, blob, tid);
         write_fresh_header<D>(blob, F, ncomp, true, tid);
     } else {
         if (tid == 0) {
@@ -770,8 +816,11 @@ __global__ void __launch_bounds__(4 * D) boundary_kernel(FlushArgs A) {
         float *So = A.S_out + head * (size_t)D * D;
         if (!s_hdr[0]) {  // unreadable blob: zeros
 #pragma unroll
-            for (int ii = 0; ii < TI; ++ii)
-                *reinterpret_cast<float4 *>(So + (size_t)(i0 + ii) * D + j0) = make_float4(0.f, 0.f, 0.f, 0.f);
+            for (int ii = 0; ii < 2 * IP; ++ii)
+#pragma unroll
+                for (int jj = 0; jj < TJ; jj += 4)
+                    *reinterpret_cast<float4 *>(So + (size_t)(i0 + ii) * D + j0 + jj) =
+                        make_float4(0.f, 0.f, 0.f, 0.f);
             return;
         }
         if (!__syncthreads_and(mbar_wait_bounded(&bar[0], 0))) {
@@ -788,16 +837,21 @@ __global__ void __launch_bounds__(4 * D) boundary_kernel(FlushArgs A) {
             __syncthreads();
             c8 = codes8;
         }
-        reconstruct_tile<D>(R, st + L.qs_off, st + L.sm_off,
+        reconstruct_tile<D>(P, st + L.qs_off, st + L.sm_off,
                             reinterpret_cast<const float *>(st + L.cvec_off), c8,
                             reinterpret_cast<const float *>(st + L.pairs_off),
                             F.kda ? reinterpret_cast<const float *>(st + L.g_off) : nullptr, H.g,
                             reinterpret_cast<const uint32_t *>(st + kHdrMeta), (int)H.ncomp,
                             (int)H.count, F.f16_scale, tid);
 #pragma unroll
-        for (int ii = 0; ii < TI; ++ii)
-            *reinterpret_cast<float4 *>(So + (size_t)(i0 + ii) * D + j0) =
-                make_float4(R[ii][0], R[ii][1], R[ii][2], R[ii][3]);
+        for (int ip = 0; ip < IP; ++ip)
+#pragma unroll
+            for (int jj = 0; jj < TJ; jj += 4) {
+                *reinterpret_cast<float4 *>(So + (size_t)(i0 + 2 * ip) * D + j0 + jj) =
+                    make_float4(P[ip][jj].x, P[ip][jj + 1].x, P[ip][jj + 2].x, P[ip][jj + 3].x);
+                *reinterpret_cast<float4 *>(So + (size_t)(i0 + 2 * ip + 1) * D + j0 + jj) =
+                    make_float4(P[ip][jj].y, P[ip][jj + 1].y, P[ip][jj + 2].y, P[ip][jj + 3].y);
+            }
     }
 }
 
