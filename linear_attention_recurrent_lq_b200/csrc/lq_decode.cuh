@@ -28,11 +28,11 @@
 //    chunk to int16 with the chunk's own scale (error <= 2^-16 of the chunk's
 //    largest entry) and dp2a multiplies two int16 entries by two int8 codes,
 //    accumulating exactly in int32;
-//  * a row is split over D/16 threads (one chunk each); a reduce-scatter over
-//    them leaves each thread with (a_j, b_j) of one row j, to which it adds
-//    the compensator and pair terms from shared memory before forming u_j and
-//    o_j.  Waits on the ring sleep on the mbarrier and give up after a bounded
-//    time.
+//  * a row is split over D/16 threads (one chunk each); the chunk sums meet in
+//    shared memory, where thread j adds up row j and then the compensator and
+//    pair terms before forming u_j and o_j.  Waits on the ring sleep on the
+//    mbarrier and give up after a bounded time; a consumer warp hands the
+//    stage back as soon as it is done with it.
 #pragma once
 
 #include "lq_common.cuh"
@@ -70,11 +70,11 @@ __host__ __device__ inline DecodeStage decode_stage(const Layout &L, int D, int 
 
 template <int D>
 __host__ __device__ constexpr uint32_t decode_fixed_smem() {
-    // barriers + control (128) | y [2D] | X int16 [2D] | chunk scales [2*D/16] | dots [2*kDotSlots]
-    // | column terms [2D] | new keys [D] | new decay [D] | reduce [32] | producer batch [3*32]
-    // | comp lists [2*16] | info [8]
-    return align_up(128u + (2u * D + D + 2u * (D / 16) + 2u * kDotSlots + 2u * D + 2u * D + 32u +
-                            96u + 32u + 8u) * 4u, 128u);
+    // barriers + control (128) | chunk sums float2 [D/16][D+1] | y [2D] | X int16 [2D]
+    // | chunk scales [2*D/16] | dots float2 [kDotSlots] | column terms float2 [D] | new keys [D]
+    // | new decay [D] | reduce [32] | producer batch [3*32] | comp lists [2*16] | info [8]
+    return align_up(128u + (2u * (D / 16) * (D + 1) + 2u * D + D + 2u * (D / 16) + 2u * kDotSlots + 2u * D +
+                            2u * D + 32u + 96u + 32u + 8u) * 4u, 128u);
 }
 
 constexpr int kDecodeStages = 2;
@@ -211,22 +211,12 @@ __device__ __forceinline__ void group_dot(const Group<BITS> &g, const uint32_t (
     }
 }
 
-// Reduce-scatter of N float2 values over N consecutive lanes of an aligned
-// group (N a power of two <= 32): afterwards lane l holds the group sum of
-// value (l mod N) in v[0].
-template <int N>
-__device__ __forceinline__ void reduce_scatter2(float2 (&v)[N], int lane) {
-#pragma unroll
-    for (int off = N / 2; off >= 1; off >>= 1) {
-        const bool upper = (lane & off) != 0;
-#pragma unroll
-        for (int i = 0; i < off; ++i) {
-            const float2 send = upper ? v[i] : v[i + off];
-            const float2 keep = upper ? v[i + off] : v[i];
-            v[i].x = keep.x + __shfl_xor_sync(0xFFFFFFFFu, send.x, off);
-            v[i].y = keep.y + __shfl_xor_sync(0xFFFFFFFFu, send.y, off);
-        }
-    }
+// Approximate reciprocal (one MUFU op, relative error below 2^-22 for
+// normal x; subnormal results flush to zero).
+__device__ __forceinline__ float rcp_approx(float x) {
+    float r;
+    asm("rcp.approx.ftz.f32 %0, %1;" : "=f"(r) : "f"(x));
+    return r;
 }
 
 __device__ __forceinline__ float warp_sum(float x) {
@@ -242,8 +232,9 @@ __global__ void __launch_bounds__(D + 32) decode_kernel(DecodeArgs A) {
     constexpr int RPT = D / 16;      // rows per thread (16 row groups)
     constexpr int GB = group_bytes<BITS>();
     constexpr int NCH = D / 16;      // chunks per row
-    constexpr int KPL = D / 16;      // keys per thread in the dot-product phase
-    constexpr int NJ = NC / 16;      // dot-product jobs per pass
+    constexpr int KPJ = D / 8;       // keys per lane in the dot-product phase
+    constexpr int PSTR = D + 1;      // padded row of the chunk-sum array (spreads the banks)
+    constexpr int NJ = NC / 8;       // dot-product jobs per pass
     constexpr int BIAS = BITS == 8 ? 0 : (BITS == 6 ? 32 : 8);
     const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
     const Layout L = A.L;
@@ -256,12 +247,13 @@ __global__ void __launch_bounds__(D + 32) decode_kernel(DecodeArgs A) {
     uint64_t *full = reinterpret_cast<uint64_t *>(smem);  // [2]
     uint64_t *empty = full + 2;                           // [2]
     volatile uint32_t *s_abort = reinterpret_cast<volatile uint32_t *>(smem + 120);
-    float *s_y = reinterpret_cast<float *>(smem + 128);          // y_k [D] | y_q [D]
+    float2 *s_part = reinterpret_cast<float2 *>(smem + 128);     // chunk sums [LPR][PSTR]
+    float *s_y = reinterpret_cast<float *>(s_part + LPR * PSTR); // y_k [D] | y_q [D]
     int16_t *s_X = reinterpret_cast<int16_t *>(s_y + 2 * D);     // X_k [D] | X_q [D] (chunk order)
     float *s_sc = reinterpret_cast<float *>(s_X + 2 * D);        // chunk scales k [NCH] | q [NCH]
-    float *s_dot = s_sc + 2 * NCH;                               // k-side [kDotSlots] | q-side
-    float *s_cadd = s_dot + 2 * kDotSlots;                       // column-compensator terms [2][D]
-    float *s_kh = s_cadd + 2 * D;                                // new key, window-start frame [D]
+    float2 *s_dot = reinterpret_cast<float2 *>(s_sc + 2 * NCH);  // (k-side, q-side) [kDotSlots]
+    float2 *s_cadd = s_dot + kDotSlots;                          // column-compensator terms [D]
+    float *s_kh = reinterpret_cast<float *>(s_cadd + D);         // new key, window-start frame [D]
     float *s_g = s_kh + D;                                       // new decay product [D]
     float *s_red = s_g + D;                                      // [32]
     uint32_t *s_cnt = reinterpret_cast<uint32_t *>(s_red + 32);  // producer batch [32]
@@ -275,7 +267,7 @@ __global__ void __launch_bounds__(D + 32) decode_kernel(DecodeArgs A) {
     if (tid == 0) {
         for (int s = 0; s < kDecodeStages; ++s) {
             mbar_init(&full[s], 1);
-            mbar_init(&empty[s], 1);
+            mbar_init(&empty[s], NC / 32);  // one arrival per consumer warp
         }
         *s_abort = 0u;
         fence_mbar_init();
@@ -329,13 +321,11 @@ __global__ void __launch_bounds__(D + 32) decode_kernel(DecodeArgs A) {
     }
 
     // ---------------------------------------------------- consumer threads
-    // GEMV role: chunk c of rows j = RPT*rg + m (m < RPT); after the
-    // reduce-scatter this thread owns row jrow = RPT*rg + c, so a warp's rows
-    // are 32 consecutive value channels.
+    // GEMV role: chunk c of rows RPT*rg + m (m < RPT); the per-chunk sums go
+    // to shared memory and thread j then owns row j in the epilogue.
     const int c = tid % LPR, rg = tid / LPR;
-    const int jrow = RPT * rg + c;
-    // dot-product role: job slot and key chunk
-    const int djob = tid / 16, dkc = tid % 16;
+    // dot-product role: 8 lanes per job, lane kc takes keys 4*kc + 32*e + (0..3)
+    const int kc = tid % 8, jslot = tid / 8;
     const uint8_t *code_base = A.state + L.codes_off + c * GB;
 
     Group<BITS> cg[RPT];
@@ -345,6 +335,10 @@ __global__ void __launch_bounds__(D + 32) decode_kernel(DecodeArgs A) {
         for (int m = 0; m < RPT; ++m) load_group<BITS>(cg[m], cb + (size_t)(RPT * rg + m) * L.row_bytes);
     }
 
+    // Every iteration starts with a barrier over all consumers (the wait on
+    // the stage), so the scratch arrays of the previous blob are free by
+    // then; the stage itself goes back to the producer when every consumer
+    // warp has arrived on its "empty" barrier.
     for (int it = 0; it < n_mine; ++it) {
         const int s = it % kDecodeStages;
         const uint32_t ph = (uint32_t)(it / kDecodeStages) & 1u;
@@ -411,9 +405,9 @@ __global__ void __launch_bounds__(D + 32) decode_kernel(DecodeArgs A) {
             s_y[D + i] = yq;
             s_kh[i] = bad ? 0.f : __fdiv_rn(kv, gnew);  // the new key in the window-start frame
             s_g[i] = gnew;
-            s_cadd[i] = 0.f;
-            s_cadd[D + i] = 0.f;
-            // x = sm . y, quantized per 16-key chunk to int16 with the chunk's scale
+            s_cadd[i] = make_float2(0.f, 0.f);
+            // x = sm . y, quantized per 16-key chunk to int16 with scale ~32767 / (chunk max):
+            // rint(x * scale) is taken by adding 1.5 * 2^23 (the result stays below 2^22)
             const float smv = load_scale(st + L.sm_off, i, F.f16_scale);
             const float xk = smv * yk, xq = smv * yq;
             float mk = fabsf(xk), mq = fabsf(xq);
@@ -422,13 +416,17 @@ __global__ void __launch_bounds__(D + 32) decode_kernel(DecodeArgs A) {
                 mk = fmaxf(mk, __shfl_xor_sync(0xFFFFFFFFu, mk, off));
                 mq = fmaxf(mq, __shfl_xor_sync(0xFFFFFFFFu, mq, off));
             }
-            const float ik = mk > 0.f ? 32767.f / mk : 0.f, iq = mq > 0.f ? 32767.f / mq : 0.f;
+            float ik = 0.f, iq = 0.f;  // chunks below 2^-100 are dropped (contribute 0)
+            if (mk >= 0x1p-100f) ik = mk < 0x1p100f ? 32767.f * rcp_approx(mk) : __fdiv_rn(32767.f, mk);
+            if (mq >= 0x1p-100f) iq = mq < 0x1p100f ? 32767.f * rcp_approx(mq) : __fdiv_rn(32767.f, mq);
+            const float2 t = __ffma2_rn(make_float2(xk, xq), make_float2(ik, iq),
+                                        make_float2(12582912.0f, 12582912.0f));
             const int slot = (i & ~15) + xslot<BITS>(i & 15);
-            s_X[slot] = (int16_t)max(-32767, min(32767, __float2int_rn(xk * ik)));
-            s_X[D + slot] = (int16_t)max(-32767, min(32767, __float2int_rn(xq * iq)));
+            s_X[slot] = (int16_t)(__float_as_uint(t.x) & 0xFFFFu);
+            s_X[D + slot] = (int16_t)(__float_as_uint(t.y) & 0xFFFFu);
             if ((i & 15) == 0) {
-                s_sc[i >> 4] = ik > 0.f ? 1.f / ik : 0.f;
-                s_sc[NCH + (i >> 4)] = iq > 0.f ? 1.f / iq : 0.f;
+                s_sc[i >> 4] = ik > 0.f ? mk * (1.f / 32767.f) : 0.f;
+                s_sc[NCH + (i >> 4)] = iq > 0.f ? mq * (1.f / 32767.f) : 0.f;
             }
             const float kq = warp_sum(kv * qv);
             if (lane == 0) s_red[warp] = kq;
@@ -449,49 +447,36 @@ __global__ void __launch_bounds__(D + 32) decode_kernel(DecodeArgs A) {
             const uint32_t *meta = reinterpret_cast<const uint32_t *>(st + kHdrMeta);
             // ---- dot products of buffered keys / compensator columns with y
             const int jobs = (int)count + ncol;
-            if (jobs > 0) {
-                float yk[KPL], yq[KPL];
+            for (int jb0 = 0; jb0 < jobs; jb0 += NJ) {
+                const int jb = jb0 + jslot;
+                const bool live = jb < jobs;
+                float2 ak2 = make_float2(0.f, 0.f), aq2 = make_float2(0.f, 0.f);
+                if (live) {
+                    const float *vec = jb < (int)count ? pairs + (size_t)jb * 2 * D
+                                                       : cvec + (size_t)s_colc[jb - count] * D;
 #pragma unroll
-                for (int e = 0; e < KPL; e += 4) {
-                    const float4 a4 = *reinterpret_cast<const float4 *>(s_y + dkc * KPL + e);
-                    const float4 b4 = *reinterpret_cast<const float4 *>(s_y + D + dkc * KPL + e);
-                    yk[e] = a4.x; yk[e + 1] = a4.y; yk[e + 2] = a4.z; yk[e + 3] = a4.w;
-                    yq[e] = b4.x; yq[e + 1] = b4.y; yq[e + 2] = b4.z; yq[e + 3] = b4.w;
+                    for (int e = 0; e < KPJ / 4; ++e) {
+                        const int o = 4 * kc + 32 * e;
+                        const float4 x4 = *reinterpret_cast<const float4 *>(vec + o);
+                        const float4 a4 = *reinterpret_cast<const float4 *>(s_y + o);
+                        const float4 b4 = *reinterpret_cast<const float4 *>(s_y + D + o);
+                        ak2 = __ffma2_rn(make_float2(x4.x, x4.y), make_float2(a4.x, a4.y), ak2);
+                        ak2 = __ffma2_rn(make_float2(x4.z, x4.w), make_float2(a4.z, a4.w), ak2);
+                        aq2 = __ffma2_rn(make_float2(x4.x, x4.y), make_float2(b4.x, b4.y), aq2);
+                        aq2 = __ffma2_rn(make_float2(x4.z, x4.w), make_float2(b4.z, b4.w), aq2);
+                    }
                 }
-                for (int jb0 = 0; jb0 < jobs; jb0 += NJ) {
-                    const int jb = jb0 + djob;
-                    const bool live = jb < jobs;
-                    float dk_ = 0.f, dq_ = 0.f;
-                    if (live) {
-                        const float *vec = jb < (int)count ? pairs + (size_t)jb * 2 * D
-                                                           : cvec + (size_t)s_colc[jb - count] * D;
+                float dk_ = ak2.x + ak2.y, dq_ = aq2.x + aq2.y;
 #pragma unroll
-                        for (int e = 0; e < KPL; e += 4) {
-                            const float4 x4 = *reinterpret_cast<const float4 *>(vec + dkc * KPL + e);
-                            dk_ = fmaf(x4.x, yk[e], dk_); dk_ = fmaf(x4.y, yk[e + 1], dk_);
-                            dk_ = fmaf(x4.z, yk[e + 2], dk_); dk_ = fmaf(x4.w, yk[e + 3], dk_);
-                            dq_ = fmaf(x4.x, yq[e], dq_); dq_ = fmaf(x4.y, yq[e + 1], dq_);
-                            dq_ = fmaf(x4.z, yq[e + 2], dq_); dq_ = fmaf(x4.w, yq[e + 3], dq_);
-                        }
-                    }
-#pragma unroll
-                    for (int off = 8; off >= 1; off >>= 1) {
-                        dk_ += __shfl_xor_sync(0xFFFFFFFFu, dk_, off);
-                        dq_ += __shfl_xor_sync(0xFFFFFFFFu, dq_, off);
-                    }
-                    if (live && dkc == 0) {
-                        if (jb < (int)count) {
-                            s_dot[jb] = dk_;
-                            s_dot[kDotSlots + jb] = dq_;
-                        } else {
-                            const int j0 = (int)(meta[s_colc[jb - count]] & 0x7FFFFFFFu);
-                            s_cadd[j0] = dk_;
-                            s_cadd[D + j0] = dq_;
-                        }
-                    }
+                for (int off = 4; off >= 1; off >>= 1) {
+                    dk_ += __shfl_xor_sync(0xFFFFFFFFu, dk_, off);
+                    dq_ += __shfl_xor_sync(0xFFFFFFFFu, dq_, off);
+                }
+                if (live && kc == 0) {
+                    if (jb < (int)count) s_dot[jb] = make_float2(dk_, dq_);
+                    else s_cadd[meta[s_colc[jb - count]] & 0x7FFFFFFFu] = make_float2(dk_, dq_);
                 }
             }
-            consumer_sync(NC);
 
             // ---- fused dequantize + dual GEMV over the codes (integer pipe)
             uint32_t Xk[8], Xq[8];
@@ -504,7 +489,7 @@ __global__ void __launch_bounds__(D + 32) decode_kernel(DecodeArgs A) {
                 Xq[0] = b0.x; Xq[1] = b0.y; Xq[2] = b0.z; Xq[3] = b0.w;
                 Xq[4] = b1.x; Xq[5] = b1.y; Xq[6] = b1.z; Xq[7] = b1.w;
             }
-            const float sck = s_sc[c], scq = s_sc[NCH + c];
+            const float2 sc2 = make_float2(s_sc[c], s_sc[NCH + c]);
             int biask = 0, biasq = 0;
             if constexpr (BIAS != 0) {
 #pragma unroll
@@ -515,40 +500,39 @@ __global__ void __launch_bounds__(D + 32) decode_kernel(DecodeArgs A) {
                 biask *= BIAS;
                 biasq *= BIAS;
             }
-            float2 acc[RPT];
 #pragma unroll
             for (int m = 0; m < RPT; ++m) {
                 int ak = -biask, aq = -biasq;
                 group_dot<BITS>(cg[m], Xk, Xq, ak, aq);
                 if (has_next) load_group<BITS>(cg[m], next_codes + (size_t)(RPT * rg + m) * L.row_bytes);
-                acc[m] = make_float2((float)ak * sck, (float)aq * scq);
+                s_part[c * PSTR + RPT * rg + m] = __fmul2_rn(make_float2((float)ak, (float)aq), sc2);
             }
-            reduce_scatter2<LPR>(acc, lane);
+            consumer_sync(NC);
 
-            // ---- epilogue: this thread owns (a_j, b_j) of row j
-            const int j = jrow;
+            // ---- epilogue: thread j owns (a_j, b_j) of row j
+            const int j = tid;
+            float2 ab = s_part[j];
+#pragma unroll
+            for (int x = 1; x < LPR; ++x) ab = __fadd2_rn(ab, s_part[x * PSTR + j]);
             const float qsj = load_scale(st + L.qs_off, j, F.f16_scale);
-            float a = qsj * acc[0].x + s_cadd[j];
-            float b = qsj * acc[0].y + s_cadd[D + j];
+            ab = __ffma2_rn(ab, make_float2(qsj, qsj), s_cadd[j]);
             for (int r = 0; r < nrow; ++r) {
                 const uint32_t cc = s_rowc[r];
                 const float wj = cvec[(size_t)cc * D + j];
                 const int i0 = (int)(meta[cc] & 0x7FFFFFFFu);
-                a = fmaf(s_y[i0], wj, a);
-                b = fmaf(s_y[D + i0], wj, b);
+                ab = __ffma2_rn(make_float2(s_y[i0], s_y[D + i0]), make_float2(wj, wj), ab);
             }
             const float *up = pairs + D + j;
 #pragma unroll 4
             for (uint32_t m = 0; m < count; ++m) {
                 const float uj = up[(size_t)m * 2 * D];
-                a = fmaf(s_dot[m], uj, a);
-                b = fmaf(s_dot[kDotSlots + m], uj, b);
+                ab = __ffma2_rn(s_dot[m], make_float2(uj, uj), ab);
             }
-            const float u = aux[0] * (load_in(qkv + 2 * SG.qkv_bytes, j, F.bf16_in) - a);
+            const float u = aux[0] * (load_in(qkv + 2 * SG.qkv_bytes, j, F.bf16_in) - ab.x);
             float kq = 0.f;
 #pragma unroll
             for (int w = 0; w < NC / 32; ++w) kq += s_red[w];
-            A.out[h * D + j] = fmaf(kq, u, b);
+            A.out[h * D + j] = fmaf(kq, u, ab.y);
             float *pair = reinterpret_cast<float *>(blob + L.pairs_off + (size_t)count * L.pair_bytes);
             pair[D + j] = u;
             pair[tid] = s_kh[tid];
@@ -566,8 +550,8 @@ __global__ void __launch_bounds__(D + 32) decode_kernel(DecodeArgs A) {
             A.out[h * D + tid] = 0.f;
             if (tid == 0 && newbits) set_status(blob, newbits);
         }
-        consumer_sync(NC);  // every consumer is done with stage s and the scratch
-        if (tid == 0) mbar_arrive(&empty[s]);
+        __syncwarp();
+        if (lane == 0) mbar_arrive(&empty[s]);  // this warp is done with stage s
     }
 }
 
