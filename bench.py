@@ -193,6 +193,28 @@ def dist_setup():
     return world, rank, local
 
 
+def max_over_ranks(vals, torch, dist, world, device):
+    """Element-wise maximum of a list of times over all ranks (the job takes
+    as long as its slowest rank); the identity on one rank."""
+    if world <= 1:
+        return [float(v) for v in vals]
+    t = torch.tensor([float(v) for v in vals], device=device, dtype=torch.float64)
+    dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    return t.tolist()
+
+
+def rank_workload(wl, rank):
+    """Each rank runs its own independent sequences (weak scaling: replicas,
+    no exchange between ranks): same shapes, another seed."""
+    return wl if rank == 0 else wl.replace(seed=wl.seed + 1000 * rank)
+
+
+def whole_job_rate(units_per_rank, world, ms):
+    """Units per second of the whole job: every rank's units over the
+    slowest rank's time."""
+    return units_per_rank * world / (ms / 1e3)
+
+
 # ------------------------------------------------------------ our arm
 
 class Arm:
@@ -280,10 +302,7 @@ def time_arm(arm, steps, warmup, torch, dist, world):
     total = start.elapsed_time(end)
     dec = sum(a.elapsed_time(b) for a, b, _ in marks)
     fl = sum(b.elapsed_time(c) for _, b, c in marks)
-    if world > 1:
-        t = torch.tensor([total, dec, fl], device="cuda", dtype=torch.float64)
-        dist.all_reduce(t, op=dist.ReduceOp.MAX)
-        total, dec, fl = t.tolist()
+    total, dec, fl = max_over_ranks([total, dec, fl], torch, dist, world, "cuda")
     return total, dec, fl
 
 
@@ -316,11 +335,7 @@ def time_e2e(arm, host, steps, torch, dist, world):
     torch.cuda.synchronize()
     if world > 1:
         dist.barrier()
-    ms = start.elapsed_time(end)
-    if world > 1:
-        t = torch.tensor([ms], device="cuda", dtype=torch.float64)
-        dist.all_reduce(t, op=dist.ReduceOp.MAX)
-        ms = t.item()
+    ms = max_over_ranks([start.elapsed_time(end)], torch, dist, world, "cuda")[0]
     return ms, h2d, d2h
 
 
@@ -396,9 +411,7 @@ def main_ours(args):
     from linear_attention_recurrent_lq_b200 import binding as B
     from linear_attention_recurrent_lq_b200 import inputs as I
 
-    wl = I.WORKLOADS[args.workload]
-    if rank:
-        wl = wl.replace(seed=wl.seed + 1000 * rank)  # other sequences on other ranks
+    wl = rank_workload(I.WORKLOADS[args.workload], rank)
     L = args.layers
     layers = make_layers(wl, L, torch, I)
     peaks, peak_kind = measured_peaks()
@@ -418,8 +431,7 @@ def main_ours(args):
     if status != 0:
         raise RuntimeError(f"device status after timing: {B.STATUS_NAMES[status]}")
     W = wl.window
-    head_tokens = args.steps * W * L * nh * world
-    value = head_tokens / (total / 1e3)
+    value = whole_job_rate(args.steps * W * L * nh, world, total)
     dec_launches = args.steps * W * L
     dec_bytes_per_launch = nh * sum(decode_bytes(wl, c) for c in range(W)) / W
     dec_ms = dec / dec_launches
@@ -454,7 +466,7 @@ def main_ours(args):
         arm32.capture()
         ks = args.fp32_steps or max(4, args.steps // 4)
         t32, d32, _ = time_arm(arm32, ks, max(3, args.warmup // 2), torch, dist, world)
-        v32 = ks * W * L * nh * world / (t32 / 1e3)
+        v32 = whole_job_rate(ks * W * L * nh, world, t32)
         b32 = nh * fp32_bytes(wl)
         a32 = b32 / (d32 / (ks * W * L) / 1e3) / 1e9
         line["fp32_state"] = {"value": v32, "unit": "head-tokens/s", "steps": ks,
@@ -472,7 +484,7 @@ def main_ours(args):
             host.append({"in": hin, "out": torch.empty_like(arm.out[l], device="cpu").pin_memory()})
         ke = args.e2e_steps or max(3, args.steps // 10)
         ms, h2d, d2h = time_e2e(arm, host, ke, torch, dist, world)
-        line["e2e"] = {"value": ke * W * L * nh * world / (ms / 1e3), "unit": "head-tokens/s",
+        line["e2e"] = {"value": whole_job_rate(ke * W * L * nh, world, ms), "unit": "head-tokens/s",
                        "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h,
                        "steps": ke, "ms_per_step": ms / ke}
 
