@@ -98,7 +98,7 @@ lq_status launch_decode(const lq_config &c, const DecodeArgs &a, cudaStream_t s)
     auto k = decode_kernel<D, BITS>;
     cudaError_t e = allow_smem(k, smem);
     if (e != cudaSuccess) return LQ_ERR_CUDA;
-    const int threads = D + 32;
+    const int threads = D + 64;
     const int grid = persistent_grid(k, threads, smem, a.num_heads);
     if (grid <= 0) return LQ_ERR_CUDA;
     k<<<grid, threads, smem, s>>>(a);

@@ -68,13 +68,25 @@ __host__ __device__ inline DecodeStage decode_stage(const Layout &L, int D, int 
     return S;
 }
 
+// Per-head scratch written by the prep warp one head ahead of the consumers
+// (two of them, by head parity):
+//   y [2D] f32 | X [2D] int16 | chunk scales [2*D/16] | khat [D] | g [D]
+//   | column terms float2 [D] | row / column compensator lists [2*16] | info [8]
+template <int D>
+struct PrepBuf {
+    static constexpr uint32_t y = 0, X = 8 * D, sc = 12 * D, kh = sc + 8 * (D / 16), g = kh + 4 * D,
+                              cadd = g + 4 * D, rowc = cadd + 8 * D, colc = rowc + 64, info = colc + 64,
+                              bytes = info + 32;
+};
+// info words
+constexpr int kInfoRun = 0, kInfoCount = 1, kInfoNrow = 2, kInfoNcol = 3, kInfoBits = 4, kInfoKq = 5;
+
 template <int D>
 __host__ __device__ constexpr uint32_t decode_fixed_smem() {
-    // barriers + control (128) | chunk sums float2 [D/16][D+1] | y [2D] | X int16 [2D]
-    // | chunk scales [2*D/16] | dots float2 [kDotSlots] | column terms float2 [D] | new keys [D]
-    // | new decay [D] | reduce [32] | producer batch [3*32] | comp lists [2*16] | info [8]
-    return align_up(128u + (2u * (D / 16) * (D + 1) + 2u * D + D + 2u * (D / 16) + 2u * kDotSlots + 2u * D +
-                            2u * D + 32u + 96u + 32u + 8u) * 4u, 128u);
+    // barriers + control (128) | chunk sums float2 [D/16][D+1] | prep buffers [2]
+    // | dots float2 [kDotSlots] | producer batch [3*32]
+    return align_up(128u + 8u * (D / 16) * (D + 1) + 2u * PrepBuf<D>::bytes + 8u * kDotSlots + 3u * 32u * 4u,
+                    128u);
 }
 
 constexpr int kDecodeStages = 2;
@@ -226,7 +238,7 @@ __device__ __forceinline__ float warp_sum(float x) {
 }
 
 template <int D, int BITS>
-__global__ void __launch_bounds__(D + 32) decode_kernel(DecodeArgs A) {
+__global__ void __launch_bounds__(D + 64) decode_kernel(DecodeArgs A) {
     constexpr int NC = D;            // consumer threads
     constexpr int LPR = D / 16;      // threads per row, one 16-key chunk each
     constexpr int RPT = D / 16;      // rows per thread (16 row groups)
@@ -235,7 +247,11 @@ __global__ void __launch_bounds__(D + 32) decode_kernel(DecodeArgs A) {
     constexpr int KPJ = D / 8;       // keys per lane in the dot-product phase
     constexpr int PSTR = D + 1;      // padded row of the chunk-sum array (spreads the banks)
     constexpr int NJ = NC / 8;       // dot-product jobs per pass
+    constexpr int KPL = D / 32;      // keys per lane of the prep warp
+    constexpr int LPC = 16 / KPL;    // prep lanes per 16-key chunk
     constexpr int BIAS = BITS == 8 ? 0 : (BITS == 6 ? 32 : 8);
+    constexpr int COPY_WARP = NC / 32, PREP_WARP = NC / 32 + 1;
+    using PB = PrepBuf<D>;
     const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
     const Layout L = A.L;
     const Flags F = A.F;
@@ -244,38 +260,31 @@ __global__ void __launch_bounds__(D + 32) decode_kernel(DecodeArgs A) {
     const int n_mine = (A.num_heads - (int)blockIdx.x + G - 1) / G;
 
     extern __shared__ __align__(128) uint8_t smem[];
-    uint64_t *full = reinterpret_cast<uint64_t *>(smem);  // [2]
-    uint64_t *empty = full + 2;                           // [2]
+    uint64_t *full = reinterpret_cast<uint64_t *>(smem);  // [2] stage landed
+    uint64_t *empty = full + 2;                           // [2] consumers done with the stage
+    uint64_t *pfull = empty + 2;                          // [2] prep of the head done
     volatile uint32_t *s_abort = reinterpret_cast<volatile uint32_t *>(smem + 120);
-    float2 *s_part = reinterpret_cast<float2 *>(smem + 128);     // chunk sums [LPR][PSTR]
-    float *s_y = reinterpret_cast<float *>(s_part + LPR * PSTR); // y_k [D] | y_q [D]
-    int16_t *s_X = reinterpret_cast<int16_t *>(s_y + 2 * D);     // X_k [D] | X_q [D] (chunk order)
-    float *s_sc = reinterpret_cast<float *>(s_X + 2 * D);        // chunk scales k [NCH] | q [NCH]
-    float2 *s_dot = reinterpret_cast<float2 *>(s_sc + 2 * NCH);  // (k-side, q-side) [kDotSlots]
-    float2 *s_cadd = s_dot + kDotSlots;                          // column-compensator terms [D]
-    float *s_kh = reinterpret_cast<float *>(s_cadd + D);         // new key, window-start frame [D]
-    float *s_g = s_kh + D;                                       // new decay product [D]
-    float *s_red = s_g + D;                                      // [32]
-    uint32_t *s_cnt = reinterpret_cast<uint32_t *>(s_red + 32);  // producer batch [32]
+    float2 *s_part = reinterpret_cast<float2 *>(smem + 128);            // chunk sums [LPR][PSTR]
+    uint8_t *s_pb = reinterpret_cast<uint8_t *>(s_part + LPR * PSTR);    // PrepBuf [2]
+    float2 *s_dot = reinterpret_cast<float2 *>(s_pb + 2 * PB::bytes);    // (k-side, q-side) [kDotSlots]
+    uint32_t *s_cnt = reinterpret_cast<uint32_t *>(s_dot + kDotSlots);  // copy-warp batch [32]
     float *s_pbeta = reinterpret_cast<float *>(s_cnt + 32);
     float *s_palpha = s_pbeta + 32;
-    uint32_t *s_rowc = reinterpret_cast<uint32_t *>(s_palpha + 32);  // key-row compensators [16]
-    uint32_t *s_colc = s_rowc + 16;                                  // value-column compensators [16]
-    uint32_t *s_info = s_colc + 16;                                  // run, count, nrow, ncol, newbits
     uint8_t *stages = smem + decode_fixed_smem<D>();
 
     if (tid == 0) {
         for (int s = 0; s < kDecodeStages; ++s) {
             mbar_init(&full[s], 1);
             mbar_init(&empty[s], NC / 32);  // one arrival per consumer warp
+            mbar_init(&pfull[s], 32);       // every lane of the prep warp
         }
         *s_abort = 0u;
         fence_mbar_init();
     }
     __syncthreads();
 
-    if (warp == NC / 32) {
-        // ------------------------------------------------ producer warp
+    if (warp == COPY_WARP) {
+        // ------------------------------------------------ copy warp
         for (int base = 0; base < n_mine; base += 32) {
             const int i = base + lane;
             if (i < n_mine) {
@@ -320,6 +329,142 @@ __global__ void __launch_bounds__(D + 32) decode_kernel(DecodeArgs A) {
         return;
     }
 
+    if (warp == PREP_WARP) {
+        // ------------------------------------------------ prep warp
+        // Per head, as soon as its stage lands: header checks, compensator
+        // lists, the new decay product, y = g . k and g . q, the new key in
+        // the window-start frame, x = sm . y quantized per 16-key chunk to
+        // int16, and k . q.  Lane l takes keys KPL*l .. KPL*l + KPL - 1.
+        for (int it = 0; it < n_mine; ++it) {
+            const int s = it % kDecodeStages;
+            const uint8_t *st = stages + (size_t)s * SG.bytes;
+            uint8_t *pb = s_pb + (it & 1) * PB::bytes;
+            uint32_t *info = reinterpret_cast<uint32_t *>(pb + PB::info);
+            if (!mbar_wait_bounded(&full[s], (uint32_t)(it / kDecodeStages) & 1u)) {
+                if (lane == 0) *s_abort = 1u;
+                break;  // the consumers time out on their own wait
+            }
+            const uint4 hdr = *reinterpret_cast<const uint4 *>(st);  // count, status, ncomp, magic
+            const uint32_t ncomp = hdr.z;
+            const bool inl = lane < (int)min(ncomp, (uint32_t)kMaxComp);
+            const uint32_t m = inl ? reinterpret_cast<const uint32_t *>(st + kHdrMeta)[lane] : 0u;
+            const bool iscol = inl && (m & kCompCol), isrow = inl && !(m & kCompCol);
+            const unsigned colm = __ballot_sync(0xFFFFFFFFu, iscol);
+            const unsigned rowm = __ballot_sync(0xFFFFFFFFu, isrow);
+            const unsigned badm = __ballot_sync(0xFFFFFFFFu, inl && (m & 0x7FFFFFFFu) >= (uint32_t)D);
+            const unsigned lt = (1u << lane) - 1u;
+            if (iscol) reinterpret_cast<uint32_t *>(pb + PB::colc)[__popc(colm & lt)] = (uint32_t)lane;
+            if (isrow) reinterpret_cast<uint32_t *>(pb + PB::rowc)[__popc(rowm & lt)] = (uint32_t)lane;
+            uint32_t newbits = 0;
+            if (hdr.w != kMagic || ncomp > (uint32_t)F.num_comp || hdr.x > (uint32_t)F.window || badm)
+                newbits = LQ_DEV_CORRUPT;
+            else if (hdr.y == 0 && hdr.x >= (uint32_t)F.window)
+                newbits = LQ_DEV_WINDOW_FULL;
+            bool run = hdr.y == 0 && newbits == 0;
+            float kq = 0.f;
+            if (run) {
+                const int i0 = KPL * lane;
+                float kv[KPL], qv[KPL], gn[KPL];
+#pragma unroll
+                for (int e = 0; e < KPL; ++e) {
+                    kv[e] = load_in(st + SG.in_off + SG.qkv_bytes, i0 + e, F.bf16_in);
+                    qv[e] = load_in(st + SG.in_off, i0 + e, F.bf16_in);
+                }
+                if (F.kda) {
+#pragma unroll
+                    for (int e = 0; e < KPL; ++e)
+                        gn[e] = reinterpret_cast<const float *>(st + L.g_off)[i0 + e] *
+                                reinterpret_cast<const float *>(st + SG.dec_off)[i0 + e];
+                } else {
+                    const float gs = *reinterpret_cast<const float *>(st + kHdrG) *
+                                     reinterpret_cast<const float *>(st + SG.aux_off)[1];
+#pragma unroll
+                    for (int e = 0; e < KPL; ++e) gn[e] = gs;
+                }
+                bool bad = false;
+                float yk[KPL], yq[KPL], kh[KPL], xk[KPL], xq[KPL];
+                float mk = 0.f, mq = 0.f;
+#pragma unroll
+                for (int e = 0; e < KPL; ++e) {
+                    bad |= !(gn[e] >= kMinDecayProduct);
+                    yk[e] = gn[e] * kv[e];
+                    yq[e] = gn[e] * qv[e];
+                    const float smv = load_scale(st + L.sm_off, i0 + e, F.f16_scale);
+                    xk[e] = smv * yk[e];
+                    xq[e] = smv * yq[e];
+                    mk = fmaxf(mk, fabsf(xk[e]));
+                    mq = fmaxf(mq, fabsf(xq[e]));
+                    kq = fmaf(kv[e], qv[e], kq);
+                }
+                bad = __any_sync(0xFFFFFFFFu, bad);
+#pragma unroll
+                for (int e = 0; e < KPL; ++e) kh[e] = bad ? 0.f : __fdiv_rn(kv[e], gn[e]);  // window-start frame
+                float *py = reinterpret_cast<float *>(pb + PB::y);
+                float *pkh = reinterpret_cast<float *>(pb + PB::kh);
+                float *pg = reinterpret_cast<float *>(pb + PB::g);
+                float2 *pcadd = reinterpret_cast<float2 *>(pb + PB::cadd);
+                if constexpr (KPL == 4) {
+                    *reinterpret_cast<float4 *>(py + i0) = make_float4(yk[0], yk[1], yk[2], yk[3]);
+                    *reinterpret_cast<float4 *>(py + D + i0) = make_float4(yq[0], yq[1], yq[2], yq[3]);
+                    *reinterpret_cast<float4 *>(pkh + i0) = make_float4(kh[0], kh[1], kh[2], kh[3]);
+                    *reinterpret_cast<float4 *>(pg + i0) = make_float4(gn[0], gn[1], gn[2], gn[3]);
+                } else {
+#pragma unroll
+                    for (int e = 0; e < KPL; ++e) {
+                        py[i0 + e] = yk[e];
+                        py[D + i0 + e] = yq[e];
+                        pkh[i0 + e] = kh[e];
+                        pg[i0 + e] = gn[e];
+                    }
+                }
+#pragma unroll
+                for (int e = 0; e < KPL; ++e) pcadd[i0 + e] = make_float2(0.f, 0.f);
+                // chunk maxima over the LPC lanes of a chunk
+#pragma unroll
+                for (int off = LPC / 2; off >= 1; off >>= 1) {
+                    mk = fmaxf(mk, __shfl_xor_sync(0xFFFFFFFFu, mk, off));
+                    mq = fmaxf(mq, __shfl_xor_sync(0xFFFFFFFFu, mq, off));
+                }
+                // int16 with scale ~32767 / (chunk max): rint(x * scale) by adding
+                // 1.5 * 2^23 (the result stays below 2^22); chunks below 2^-100
+                // are dropped (they contribute 0)
+                float ik = 0.f, iq = 0.f;
+                if (mk >= 0x1p-100f) ik = mk < 0x1p100f ? 32767.f * rcp_approx(mk) : __fdiv_rn(32767.f, mk);
+                if (mq >= 0x1p-100f) iq = mq < 0x1p100f ? 32767.f * rcp_approx(mq) : __fdiv_rn(32767.f, mq);
+                int16_t *pX = reinterpret_cast<int16_t *>(pb + PB::X);
+#pragma unroll
+                for (int e = 0; e < KPL; ++e) {
+                    const float2 t = __ffma2_rn(make_float2(xk[e], xq[e]), make_float2(ik, iq),
+                                                make_float2(12582912.0f, 12582912.0f));
+                    const int i = i0 + e, slot = (i & ~15) + xslot<BITS>(i & 15);
+                    pX[slot] = (int16_t)(__float_as_uint(t.x) & 0xFFFFu);
+                    pX[D + slot] = (int16_t)(__float_as_uint(t.y) & 0xFFFFu);
+                }
+                if (lane % LPC == 0) {
+                    float *psc = reinterpret_cast<float *>(pb + PB::sc);
+                    psc[lane / LPC] = ik > 0.f ? mk * (1.f / 32767.f) : 0.f;
+                    psc[NCH + lane / LPC] = iq > 0.f ? mq * (1.f / 32767.f) : 0.f;
+                }
+                kq = warp_sum(kq);
+                if (bad) {
+                    run = false;
+                    newbits = LQ_DEV_RANGE;
+                }
+            }
+            if (lane == 0) {
+                info[kInfoRun] = run ? 1u : 0u;
+                info[kInfoCount] = hdr.x;
+                info[kInfoNrow] = (uint32_t)__popc(rowm);
+                info[kInfoNcol] = (uint32_t)__popc(colm);
+                info[kInfoBits] = newbits;
+                info[kInfoKq] = __float_as_uint(kq);
+            }
+            __syncwarp();
+            mbar_arrive(&pfull[s]);
+        }
+        return;
+    }
+
     // ---------------------------------------------------- consumer threads
     // GEMV role: chunk c of rows RPT*rg + m (m < RPT); the per-chunk sums go
     // to shared memory and thread j then owns row j in the epilogue.
@@ -336,19 +481,20 @@ __global__ void __launch_bounds__(D + 32) decode_kernel(DecodeArgs A) {
     }
 
     // Every iteration starts with a barrier over all consumers (the wait on
-    // the stage), so the scratch arrays of the previous blob are free by
-    // then; the stage itself goes back to the producer when every consumer
-    // warp has arrived on its "empty" barrier.
+    // the prep of the head), so the chunk sums and dot products of the
+    // previous head are free by then; the stage goes back to the copy warp
+    // when every consumer warp has arrived on its "empty" barrier.
     for (int it = 0; it < n_mine; ++it) {
         const int s = it % kDecodeStages;
         const uint32_t ph = (uint32_t)(it / kDecodeStages) & 1u;
         const uint8_t *st = stages + (size_t)s * SG.bytes;
+        const uint8_t *pb = s_pb + (it & 1) * PB::bytes;
         const size_t h = blockIdx.x + (size_t)it * G;
         uint8_t *blob = A.state + h * L.blob;
         const bool has_next = it + 1 < n_mine;
         const uint8_t *next_codes = code_base + (h + G) * (size_t)L.blob;
-        if (!consumer_sync_and(mbar_wait_bounded(&full[s], ph), NC)) {
-            // the copy never completed: record it on this blob and stop this CTA
+        if (!consumer_sync_and(mbar_wait_bounded(&pfull[s], ph), NC)) {
+            // the data never arrived: record it on this blob and stop this CTA
             if (tid == 0) {
                 set_status(blob, LQ_DEV_TIMEOUT);
                 *s_abort = 1u;
@@ -356,95 +502,21 @@ __global__ void __launch_bounds__(D + 32) decode_kernel(DecodeArgs A) {
             A.out[h * D + tid] = 0.f;
             break;
         }
-        const float *aux = reinterpret_cast<const float *>(st + SG.aux_off);
-        const uint8_t *qkv = st + SG.in_off;
-
-        if (warp == 0) {
-            // header checks and compensator lists (one warp, ballots)
-            const uint4 hdr = *reinterpret_cast<const uint4 *>(st);  // count, status, ncomp, magic
-            const uint32_t ncomp = hdr.z;
-            const bool inl = lane < (int)min(ncomp, (uint32_t)kMaxComp);
-            const uint32_t m = inl ? reinterpret_cast<const uint32_t *>(st + kHdrMeta)[lane] : 0u;
-            const bool iscol = inl && (m & kCompCol), isrow = inl && !(m & kCompCol);
-            const unsigned colm = __ballot_sync(0xFFFFFFFFu, iscol);
-            const unsigned rowm = __ballot_sync(0xFFFFFFFFu, isrow);
-            const unsigned badm = __ballot_sync(0xFFFFFFFFu, inl && (m & 0x7FFFFFFFu) >= (uint32_t)D);
-            const unsigned lt = (1u << lane) - 1u;
-            if (iscol) s_colc[__popc(colm & lt)] = (uint32_t)lane;
-            if (isrow) s_rowc[__popc(rowm & lt)] = (uint32_t)lane;
-            if (lane == 0) {
-                uint32_t newbits = 0;
-                if (hdr.w != kMagic || ncomp > (uint32_t)F.num_comp || hdr.x > (uint32_t)F.window || badm)
-                    newbits = LQ_DEV_CORRUPT;
-                else if (hdr.y == 0 && hdr.x >= (uint32_t)F.window)
-                    newbits = LQ_DEV_WINDOW_FULL;
-                s_info[0] = (hdr.y == 0 && newbits == 0) ? 1u : 0u;
-                s_info[1] = hdr.x;
-                s_info[2] = (uint32_t)__popc(rowm);
-                s_info[3] = (uint32_t)__popc(colm);
-                s_info[4] = newbits;
-            }
-        }
-        bool bad;
-        {
-            const int i = tid;
-            const float kv = load_in(qkv + SG.qkv_bytes, i, F.bf16_in);
-            const float qv = load_in(qkv, i, F.bf16_in);
-            float a, gold;
-            if (F.kda) {
-                a = reinterpret_cast<const float *>(st + SG.dec_off)[i];
-                gold = reinterpret_cast<const float *>(st + L.g_off)[i];
-            } else {
-                a = aux[1];
-                gold = *reinterpret_cast<const float *>(st + kHdrG);
-            }
-            const float gnew = gold * a;
-            bad = !(gnew >= kMinDecayProduct);
-            const float yk = gnew * kv, yq = gnew * qv;
-            s_y[i] = yk;
-            s_y[D + i] = yq;
-            s_kh[i] = bad ? 0.f : __fdiv_rn(kv, gnew);  // the new key in the window-start frame
-            s_g[i] = gnew;
-            s_cadd[i] = make_float2(0.f, 0.f);
-            // x = sm . y, quantized per 16-key chunk to int16 with scale ~32767 / (chunk max):
-            // rint(x * scale) is taken by adding 1.5 * 2^23 (the result stays below 2^22)
-            const float smv = load_scale(st + L.sm_off, i, F.f16_scale);
-            const float xk = smv * yk, xq = smv * yq;
-            float mk = fabsf(xk), mq = fabsf(xq);
-#pragma unroll
-            for (int off = 8; off >= 1; off >>= 1) {
-                mk = fmaxf(mk, __shfl_xor_sync(0xFFFFFFFFu, mk, off));
-                mq = fmaxf(mq, __shfl_xor_sync(0xFFFFFFFFu, mq, off));
-            }
-            float ik = 0.f, iq = 0.f;  // chunks below 2^-100 are dropped (contribute 0)
-            if (mk >= 0x1p-100f) ik = mk < 0x1p100f ? 32767.f * rcp_approx(mk) : __fdiv_rn(32767.f, mk);
-            if (mq >= 0x1p-100f) iq = mq < 0x1p100f ? 32767.f * rcp_approx(mq) : __fdiv_rn(32767.f, mq);
-            const float2 t = __ffma2_rn(make_float2(xk, xq), make_float2(ik, iq),
-                                        make_float2(12582912.0f, 12582912.0f));
-            const int slot = (i & ~15) + xslot<BITS>(i & 15);
-            s_X[slot] = (int16_t)(__float_as_uint(t.x) & 0xFFFFu);
-            s_X[D + slot] = (int16_t)(__float_as_uint(t.y) & 0xFFFFu);
-            if ((i & 15) == 0) {
-                s_sc[i >> 4] = ik > 0.f ? mk * (1.f / 32767.f) : 0.f;
-                s_sc[NCH + (i >> 4)] = iq > 0.f ? mq * (1.f / 32767.f) : 0.f;
-            }
-            const float kq = warp_sum(kv * qv);
-            if (lane == 0) s_red[warp] = kq;
-        }
-        const bool any_bad = consumer_sync_or(bad, NC);
-        bool run = s_info[0] != 0u;
-        const uint32_t count = s_info[1];
-        const int nrow = (int)s_info[2], ncol = (int)s_info[3];
-        uint32_t newbits = s_info[4];
-        if (run && any_bad) {
-            run = false;
-            newbits = LQ_DEV_RANGE;
-        }
+        const uint32_t *info = reinterpret_cast<const uint32_t *>(pb + PB::info);
+        const bool run = info[kInfoRun] != 0u;
+        const uint32_t count = info[kInfoCount];
+        const int nrow = (int)info[kInfoNrow], ncol = (int)info[kInfoNcol];
+        const uint32_t newbits = info[kInfoBits];
+        const float *py = reinterpret_cast<const float *>(pb + PB::y);
 
         if (run) {
+            const float *aux = reinterpret_cast<const float *>(st + SG.aux_off);
             const float *pairs = reinterpret_cast<const float *>(st + SG.pairs_at);
             const float *cvec = reinterpret_cast<const float *>(st + L.cvec_off);
             const uint32_t *meta = reinterpret_cast<const uint32_t *>(st + kHdrMeta);
+            const uint32_t *colc = reinterpret_cast<const uint32_t *>(pb + PB::colc);
+            const uint32_t *rowc = reinterpret_cast<const uint32_t *>(pb + PB::rowc);
+            float2 *cadd = reinterpret_cast<float2 *>(const_cast<uint8_t *>(pb) + PB::cadd);
             // ---- dot products of buffered keys / compensator columns with y
             const int jobs = (int)count + ncol;
             for (int jb0 = 0; jb0 < jobs; jb0 += NJ) {
@@ -453,13 +525,13 @@ __global__ void __launch_bounds__(D + 32) decode_kernel(DecodeArgs A) {
                 float2 ak2 = make_float2(0.f, 0.f), aq2 = make_float2(0.f, 0.f);
                 if (live) {
                     const float *vec = jb < (int)count ? pairs + (size_t)jb * 2 * D
-                                                       : cvec + (size_t)s_colc[jb - count] * D;
+                                                       : cvec + (size_t)colc[jb - count] * D;
 #pragma unroll
                     for (int e = 0; e < KPJ / 4; ++e) {
                         const int o = 4 * kc + 32 * e;
                         const float4 x4 = *reinterpret_cast<const float4 *>(vec + o);
-                        const float4 a4 = *reinterpret_cast<const float4 *>(s_y + o);
-                        const float4 b4 = *reinterpret_cast<const float4 *>(s_y + D + o);
+                        const float4 a4 = *reinterpret_cast<const float4 *>(py + o);
+                        const float4 b4 = *reinterpret_cast<const float4 *>(py + D + o);
                         ak2 = __ffma2_rn(make_float2(x4.x, x4.y), make_float2(a4.x, a4.y), ak2);
                         ak2 = __ffma2_rn(make_float2(x4.z, x4.w), make_float2(a4.z, a4.w), ak2);
                         aq2 = __ffma2_rn(make_float2(x4.x, x4.y), make_float2(b4.x, b4.y), aq2);
@@ -474,22 +546,23 @@ __global__ void __launch_bounds__(D + 32) decode_kernel(DecodeArgs A) {
                 }
                 if (live && kc == 0) {
                     if (jb < (int)count) s_dot[jb] = make_float2(dk_, dq_);
-                    else s_cadd[meta[s_colc[jb - count]] & 0x7FFFFFFFu] = make_float2(dk_, dq_);
+                    else cadd[meta[colc[jb - count]] & 0x7FFFFFFFu] = make_float2(dk_, dq_);
                 }
             }
 
             // ---- fused dequantize + dual GEMV over the codes (integer pipe)
             uint32_t Xk[8], Xq[8];
             {
-                const uint4 *xk4 = reinterpret_cast<const uint4 *>(s_X + 16 * c);
-                const uint4 *xq4 = reinterpret_cast<const uint4 *>(s_X + D + 16 * c);
+                const uint4 *xk4 = reinterpret_cast<const uint4 *>(pb + PB::X + 32 * c);
+                const uint4 *xq4 = reinterpret_cast<const uint4 *>(pb + PB::X + 2 * D + 32 * c);
                 const uint4 a0 = xk4[0], a1 = xk4[1], b0 = xq4[0], b1 = xq4[1];
                 Xk[0] = a0.x; Xk[1] = a0.y; Xk[2] = a0.z; Xk[3] = a0.w;
                 Xk[4] = a1.x; Xk[5] = a1.y; Xk[6] = a1.z; Xk[7] = a1.w;
                 Xq[0] = b0.x; Xq[1] = b0.y; Xq[2] = b0.z; Xq[3] = b0.w;
                 Xq[4] = b1.x; Xq[5] = b1.y; Xq[6] = b1.z; Xq[7] = b1.w;
             }
-            const float2 sc2 = make_float2(s_sc[c], s_sc[NCH + c]);
+            const float *psc = reinterpret_cast<const float *>(pb + PB::sc);
+            const float2 sc2 = make_float2(psc[c], psc[NCH + c]);
             int biask = 0, biasq = 0;
             if constexpr (BIAS != 0) {
 #pragma unroll
@@ -515,12 +588,12 @@ __global__ void __launch_bounds__(D + 32) decode_kernel(DecodeArgs A) {
 #pragma unroll
             for (int x = 1; x < LPR; ++x) ab = __fadd2_rn(ab, s_part[x * PSTR + j]);
             const float qsj = load_scale(st + L.qs_off, j, F.f16_scale);
-            ab = __ffma2_rn(ab, make_float2(qsj, qsj), s_cadd[j]);
+            ab = __ffma2_rn(ab, make_float2(qsj, qsj), cadd[j]);
             for (int r = 0; r < nrow; ++r) {
-                const uint32_t cc = s_rowc[r];
+                const uint32_t cc = rowc[r];
                 const float wj = cvec[(size_t)cc * D + j];
                 const int i0 = (int)(meta[cc] & 0x7FFFFFFFu);
-                ab = __ffma2_rn(make_float2(s_y[i0], s_y[D + i0]), make_float2(wj, wj), ab);
+                ab = __ffma2_rn(make_float2(py[i0], py[D + i0]), make_float2(wj, wj), ab);
             }
             const float *up = pairs + D + j;
 #pragma unroll 4
@@ -528,18 +601,18 @@ __global__ void __launch_bounds__(D + 32) decode_kernel(DecodeArgs A) {
                 const float uj = up[(size_t)m * 2 * D];
                 ab = __ffma2_rn(s_dot[m], make_float2(uj, uj), ab);
             }
-            const float u = aux[0] * (load_in(qkv + 2 * SG.qkv_bytes, j, F.bf16_in) - ab.x);
-            float kq = 0.f;
-#pragma unroll
-            for (int w = 0; w < NC / 32; ++w) kq += s_red[w];
+            const float u = aux[0] * (load_in(st + SG.in_off + 2 * SG.qkv_bytes, j, F.bf16_in) - ab.x);
+            const float kq = __uint_as_float(info[kInfoKq]);
             A.out[h * D + j] = fmaf(kq, u, ab.y);
+            const float *pkh = reinterpret_cast<const float *>(pb + PB::kh);
+            const float *pg = reinterpret_cast<const float *>(pb + PB::g);
             float *pair = reinterpret_cast<float *>(blob + L.pairs_off + (size_t)count * L.pair_bytes);
             pair[D + j] = u;
-            pair[tid] = s_kh[tid];
-            if (F.kda) reinterpret_cast<float *>(blob + L.g_off)[tid] = s_g[tid];
+            pair[tid] = pkh[tid];
+            if (F.kda) reinterpret_cast<float *>(blob + L.g_off)[tid] = pg[tid];
             if (tid == 0) {
                 *reinterpret_cast<uint32_t *>(blob + kHdrCount) = count + 1;
-                if (!F.kda) *reinterpret_cast<float *>(blob + kHdrG) = s_g[0];
+                if (!F.kda) *reinterpret_cast<float *>(blob + kHdrG) = pg[0];
             }
         } else {
             // skipped: still move on to the next blob's codes
