@@ -4,6 +4,7 @@
 #include <stdint.h>
 
 #include <mutex>
+#include <utility>
 #include <vector>
 
 #include "leapquant.h"
@@ -60,6 +61,25 @@ cudaError_t allow_smem(K kernel, uint32_t bytes) {
     return e;
 }
 
+// Launch with programmatic stream serialization: the kernel may start while
+// the previous kernel on the stream drains; it waits for that kernel's
+// completion (pdl_wait) before its first global-memory access.
+template <typename... KArgs, typename... Args>
+cudaError_t launch_pdl(void (*kernel)(KArgs...), int grid, int threads, uint32_t smem, cudaStream_t s,
+                       Args &&...args) {
+    cudaLaunchConfig_t cfg = {};
+    cfg.gridDim = dim3((unsigned)grid);
+    cfg.blockDim = dim3((unsigned)threads);
+    cfg.dynamicSmemBytes = smem;
+    cfg.stream = s;
+    cudaLaunchAttribute attr[1];
+    attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+    attr[0].val.programmaticStreamSerializationAllowed = 1;
+    cfg.attrs = attr;
+    cfg.numAttrs = 1;
+    return cudaLaunchKernelEx(&cfg, kernel, std::forward<Args>(args)...);
+}
+
 lq_status launched(cudaError_t e) {
     if (e != cudaSuccess) return LQ_ERR_CUDA;
     return cudaGetLastError() == cudaSuccess ? LQ_OK : LQ_ERR_CUDA;
@@ -101,8 +121,7 @@ lq_status launch_decode(const lq_config &c, const DecodeArgs &a, cudaStream_t s)
     const int threads = D + 64;
     const int grid = persistent_grid(k, threads, smem, a.num_heads);
     if (grid <= 0) return LQ_ERR_CUDA;
-    k<<<grid, threads, smem, s>>>(a);
-    return launched(cudaSuccess);
+    return launched(launch_pdl(k, grid, threads, smem, s, a));
 }
 
 template <int D, int BITS, int MODE>
@@ -115,8 +134,7 @@ lq_status launch_boundary(const lq_config &c, const FlushArgs &a, cudaStream_t s
         const int threads = kGroup;
         const int grid = persistent_grid(k, threads, smem, a.num_heads);
         if (grid <= 0) return LQ_ERR_CUDA;
-        k<<<grid, threads, smem, s>>>(a);
-        return launched(cudaSuccess);
+        return launched(launch_pdl(k, grid, threads, smem, s, a));
     }
     const uint32_t smem = boundary_smem_bytes(D, BITS, a.L, c.window);
     auto k = boundary_kernel<D, BITS, MODE == 0 ? 1 : MODE>;
@@ -141,12 +159,8 @@ lq_status dispatch_boundary(const lq_config &c, const FlushArgs &a, cudaStream_t
 
 template <int D>
 lq_status launch_fp32_decode(const lq_config &c, const Fp32Args &a, cudaStream_t s) {
-    const uint32_t smem = fp32_smem_bytes<D>();
-    auto k = fp32_decode_kernel<D>;
-    cudaError_t e = allow_smem(k, smem);
-    if (e != cudaSuccess) return LQ_ERR_CUDA;
-    k<<<(unsigned)(c.num_slots * c.num_heads), 4 * D, smem, s>>>(a);
-    return launched(cudaSuccess);
+    const int grid = a.num_heads * (D / kFp32Cols);
+    return launched(launch_pdl(fp32_decode_kernel<D>, grid, kFp32Threads, 0u, s, a));
 }
 
 template <int MODE>
@@ -203,7 +217,7 @@ lq_status lq_decode_step(const lq_config *cfg, void *state, const void *q, const
     cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
     if (c.bits == 32) {
         Fp32Args a{static_cast<uint8_t *>(state), nullptr, nullptr, L, make_flags(c), q, k, v,
-                   beta, decay, out};
+                   beta, decay, out, c.num_slots * c.num_heads};
         return c.dk == 128 ? launch_fp32_decode<128>(c, a, s) : launch_fp32_decode<64>(c, a, s);
     }
     DecodeArgs a{static_cast<uint8_t *>(state), L, make_flags(c), q, k, v, beta, decay, out,

@@ -139,6 +139,14 @@ __device__ __forceinline__ void bulk_g2s(void *smem_dst, const void *gmem_src, u
         : "memory");
 }
 
+// Programmatic dependent launch: a kernel launched with programmatic stream
+// serialization may start while the previous kernel on the stream finishes;
+// pdl_wait() blocks until that kernel has completed and its memory is
+// visible (a no-op for an ordinary launch), so every global access comes
+// after it.  pdl_trigger() lets the next such kernel start its own launch.
+__device__ __forceinline__ void pdl_wait() { asm volatile("griddepcontrol.wait;" ::: "memory"); }
+__device__ __forceinline__ void pdl_trigger() { asm volatile("griddepcontrol.launch_dependents;" ::: "memory"); }
+
 __device__ __forceinline__ void set_status(uint8_t *blob, uint32_t bits) {
     atomicOr(reinterpret_cast<unsigned int *>(blob + kHdrStatus), bits);
 }

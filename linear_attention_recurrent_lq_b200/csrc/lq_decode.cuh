@@ -282,6 +282,8 @@ __global__ void __launch_bounds__(D + 64) decode_kernel(DecodeArgs A) {
         fence_mbar_init();
     }
     __syncthreads();
+    pdl_wait();
+    pdl_trigger();
 
     if (warp == COPY_WARP) {
         // ------------------------------------------------ copy warp

@@ -702,6 +702,8 @@ __global__ void __launch_bounds__(kGroup, 2) flush_kernel(FlushArgs A) {
     uint8_t *stages = scratch + group_smem_bytes<D, BITS>();
     auto blob_at = [&](int it) { return A.state + ((size_t)blockIdx.x + (size_t)it * G) * L.blob; };
 
+    pdl_wait();
+    pdl_trigger();
     if (tid == 0) {
         for (int s = 0; s < kFlushStages; ++s) mbar_init(&full[s], 1);
         fence_mbar_init();

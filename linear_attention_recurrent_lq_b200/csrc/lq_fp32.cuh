@@ -5,22 +5,21 @@
 // compresses it to 8-bit without losing accuracy", second paragraph); the
 // library keeps it as the comparison point for throughput and accuracy.
 //
-// One CTA of 4*D threads per (slot, head): thread 0 bulk-copies the D x D
-// state into shared memory; thread t owns rows TI*(t%16).. and columns
-// 4*(t/16).. (TI = D/16), forms S' = D_t S in registers, the column sums
-// S'^T k and S'^T q go through shared memory, and the thread writes
-// S' + k u^T straight back with 16-byte stores.
+// The update separates by value column: u_j = beta (v_j - (S'^T k)_j) needs
+// only column j of S' = D_t S.  So one CTA of 128 threads takes one
+// (slot, head) and a block of 32 value columns: thread t loads rows
+// TI*(t%16).. (TI = D/16) of columns 4*(t/16).. of the block straight into
+// registers with 16-byte loads, forms S', the column sums S'^T k and S'^T q
+// meet in shared memory, and it writes S' + k u^T back with 16-byte stores.
+// Many small CTAs per SM keep the loads of several heads in flight.
 #pragma once
 
 #include "lq_common.cuh"
 
 namespace lq {
 
-template <int D>
-__host__ __device__ constexpr uint32_t fp32_smem_bytes() {
-    // bar/hdr 128 | k, q, a, u [D] | partials 2 x [16][D] | state D*D
-    return 128u + (4u * D + 32u * D) * 4u + (uint32_t)D * D * 4u;
-}
+constexpr int kFp32Cols = 32;      // value columns per CTA
+constexpr int kFp32Threads = 128;  // 16 row groups x 8 column quads
 
 struct Fp32Args {
     uint8_t *state;
@@ -31,114 +30,93 @@ struct Fp32Args {
     const void *q, *k, *v;
     const float *beta, *decay;
     float *out;
+    int num_heads;
 };
 
 template <int D>
-__global__ void __launch_bounds__(4 * D) fp32_decode_kernel(Fp32Args A) {
-    constexpr int TI = D / 16;
+__global__ void __launch_bounds__(kFp32Threads) fp32_decode_kernel(Fp32Args A) {
+    constexpr int TI = D / 16, NB = D / kFp32Cols;
+    pdl_wait();
+    pdl_trigger();
     const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
-    const int ic = tid & 15, jc = tid >> 4, i0 = TI * ic, j0 = 4 * jc;
-    const size_t head = blockIdx.x;
+    const int ic = tid & 15, jc = tid >> 4, i0 = TI * ic;
+    const size_t head = blockIdx.x / NB;
+    const int cb = blockIdx.x % NB, j0 = kFp32Cols * cb + 4 * jc;
     const Flags &F = A.F;
     uint8_t *blob = A.state + head * A.L.blob;
     float *S = reinterpret_cast<float *>(blob + kHdrBytes);
 
-    extern __shared__ __align__(128) uint8_t smem[];
-    uint64_t *bar = reinterpret_cast<uint64_t *>(smem);
-    uint32_t *s_hdr = reinterpret_cast<uint32_t *>(smem + 16);
-    float *s_k = reinterpret_cast<float *>(smem + 128);
-    float *s_q = s_k + D, *s_a = s_q + D, *s_u = s_a + D;
-    float *s_pk = s_u + D;            // [16][D]
-    float *s_pq = s_pk + 16 * D;      // [16][D]
-    float *s_S = s_pq + 16 * D;       // [D][D]
+    __shared__ float s_pk[16][kFp32Cols], s_pq[16][kFp32Cols], s_u[kFp32Cols], s_kq[kFp32Threads / 32];
 
-    if (tid == 0) {
-        const uint4 h = *reinterpret_cast<const uint4 *>(blob);
-        const bool run = h.w == kMagic && h.y == 0;
-        s_hdr[0] = run ? 1u : 0u;
-        if (h.w != kMagic && h.y == 0) set_status(blob, LQ_DEV_CORRUPT);
-        if (run) {
-            mbar_init(&bar[0], 1);
-            fence_mbar_init();
-            mbar_arrive_expect_tx(&bar[0], (uint32_t)D * D * 4u);
-            bulk_g2s(s_S, S, (uint32_t)D * D * 4u, &bar[0]);
-        }
+    const uint4 hdr = *reinterpret_cast<const uint4 *>(blob);
+    const bool run = hdr.w == kMagic && hdr.y == 0;
+    if (!run) {
+        if (tid < kFp32Cols) A.out[head * D + kFp32Cols * cb + tid] = 0.f;
+        if (hdr.w != kMagic && hdr.y == 0 && cb == 0 && tid == 0) set_status(blob, LQ_DEV_CORRUPT);
+        return;
     }
-    float vv = 0.f, kq = 0.f;
+    float4 r4[TI];
+#pragma unroll
+    for (int ii = 0; ii < TI; ++ii) r4[ii] = __ldcs(reinterpret_cast<const float4 *>(S + (size_t)(i0 + ii) * D + j0));
+    float kr[TI], qr[TI], ar[TI];
+#pragma unroll
+    for (int ii = 0; ii < TI; ++ii) {
+        const size_t o = head * D + i0 + ii;
+        kr[ii] = load_in(A.k, o, F.bf16_in);
+        qr[ii] = load_in(A.q, o, F.bf16_in);
+        ar[ii] = F.kda ? A.decay[o] : A.decay[head];
+    }
+    float kq = 0.f;
     if (tid < D) {
         const size_t o = head * D + tid;
-        const float kv = load_in(A.k, o, F.bf16_in), qv = load_in(A.q, o, F.bf16_in);
-        vv = load_in(A.v, o, F.bf16_in);
-        s_k[tid] = kv;
-        s_q[tid] = qv;
-        s_a[tid] = F.kda ? A.decay[o] : A.decay[head];
-        kq = kv * qv;
+        kq = load_in(A.k, o, F.bf16_in) * load_in(A.q, o, F.bf16_in);
     }
-    const float bt = A.beta[head];
 #pragma unroll
     for (int off = 16; off >= 1; off >>= 1) kq += __shfl_xor_sync(0xFFFFFFFFu, kq, off);
-    if (lane == 0) s_pk[warp] = kq;  // scratch until the partials are written
-    __syncthreads();
-    if (!s_hdr[0]) {
-        if (tid < D) A.out[head * D + tid] = 0.f;
-        return;
-    }
-    float kq_all = 0.f;
-#pragma unroll
-    for (int w = 0; w < D / 32; ++w) kq_all += s_pk[w];
-    if (!__syncthreads_and(mbar_wait_bounded(&bar[0], 0))) {
-        if (tid < D) A.out[head * D + tid] = 0.f;
-        if (tid == 0) {
-            set_status(blob, LQ_DEV_TIMEOUT);
-            mbar_wait_bounded(&bar[0], 0);
-        }
-        return;
-    }
+    if (lane == 0) s_kq[warp] = kq;
 
     float Sd[TI][4];
     float pk[4] = {0.f, 0.f, 0.f, 0.f}, pq[4] = {0.f, 0.f, 0.f, 0.f};
 #pragma unroll
     for (int ii = 0; ii < TI; ++ii) {
-        const int i = i0 + ii;
-        const float4 r4 = *reinterpret_cast<const float4 *>(s_S + (size_t)i * D + j0);
-        const float a = s_a[i], kk = s_k[i], qq = s_q[i];
-        Sd[ii][0] = a * r4.x; Sd[ii][1] = a * r4.y; Sd[ii][2] = a * r4.z; Sd[ii][3] = a * r4.w;
+        const float a = ar[ii];
+        Sd[ii][0] = a * r4[ii].x; Sd[ii][1] = a * r4[ii].y; Sd[ii][2] = a * r4[ii].z; Sd[ii][3] = a * r4[ii].w;
 #pragma unroll
         for (int jj = 0; jj < 4; ++jj) {
-            pk[jj] = fmaf(Sd[ii][jj], kk, pk[jj]);
-            pq[jj] = fmaf(Sd[ii][jj], qq, pq[jj]);
+            pk[jj] = fmaf(Sd[ii][jj], kr[ii], pk[jj]);
+            pq[jj] = fmaf(Sd[ii][jj], qr[ii], pq[jj]);
         }
     }
-    *reinterpret_cast<float4 *>(s_pk + ic * D + j0) = make_float4(pk[0], pk[1], pk[2], pk[3]);
-    *reinterpret_cast<float4 *>(s_pq + ic * D + j0) = make_float4(pq[0], pq[1], pq[2], pq[3]);
+    *reinterpret_cast<float4 *>(&s_pk[ic][4 * jc]) = make_float4(pk[0], pk[1], pk[2], pk[3]);
+    *reinterpret_cast<float4 *>(&s_pq[ic][4 * jc]) = make_float4(pq[0], pq[1], pq[2], pq[3]);
     __syncthreads();
-    if (tid < D) {
-        float a = 0.f, b = 0.f;
+    if (tid < kFp32Cols) {
+        float a = 0.f, b = 0.f, kq_all = 0.f;
 #pragma unroll
         for (int r = 0; r < 16; ++r) {
-            a += s_pk[r * D + tid];
-            b += s_pq[r * D + tid];
+            a += s_pk[r][tid];
+            b += s_pq[r][tid];
         }
-        const float u = bt * (vv - a);
+#pragma unroll
+        for (int w = 0; w < kFp32Threads / 32; ++w) kq_all += s_kq[w];
+        const size_t o = head * D + kFp32Cols * cb + tid;
+        const float u = A.beta[head] * (load_in(A.v, o, F.bf16_in) - a);
         s_u[tid] = u;
-        A.out[head * D + tid] = fmaf(kq_all, u, b);
+        A.out[o] = fmaf(kq_all, u, b);
     }
     __syncthreads();
-    const float4 u4 = *reinterpret_cast<const float4 *>(s_u + j0);
-    const float uu[4] = {u4.x, u4.y, u4.z, u4.w};
+    const float4 u4 = *reinterpret_cast<const float4 *>(&s_u[4 * jc]);
 #pragma unroll
     for (int ii = 0; ii < TI; ++ii) {
-        const float kk = s_k[i0 + ii];
         float4 o4;
-        o4.x = fmaf(kk, uu[0], Sd[ii][0]);
-        o4.y = fmaf(kk, uu[1], Sd[ii][1]);
-        o4.z = fmaf(kk, uu[2], Sd[ii][2]);
-        o4.w = fmaf(kk, uu[3], Sd[ii][3]);
-        *reinterpret_cast<float4 *>(S + (size_t)(i0 + ii) * D + j0) = o4;
+        o4.x = fmaf(kr[ii], u4.x, Sd[ii][0]);
+        o4.y = fmaf(kr[ii], u4.y, Sd[ii][1]);
+        o4.z = fmaf(kr[ii], u4.z, Sd[ii][2]);
+        o4.w = fmaf(kr[ii], u4.w, Sd[ii][3]);
+        __stcs(reinterpret_cast<float4 *>(S + (size_t)(i0 + ii) * D + j0), o4);
     }
 }
 
-// init (MODE 1): S0 -> blob with a fresh header; dequant (MODE 2): blob -> S_out
 template <int D, int MODE>
 __global__ void __launch_bounds__(256) fp32_copy_kernel(Fp32Args A) {
     const size_t head = blockIdx.x;
