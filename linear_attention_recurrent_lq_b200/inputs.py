@@ -98,6 +98,15 @@ WORKLOADS = {
         name="gdn_4bit_b256h32", batch=256, heads=32, tokens=1024, window=16,
         num_comp=8, bits=4, decay_kind="gdn", smoothing=True,
         scale_dtype="f16", seed=3),
+    # prefix-cache-scale layer: 48 heads mixed 3:1 GDN:KDA, held as two states
+    # (36 GDN heads and 12 KDA heads per sequence); W and r are swept
+    "mix_gdn_b512h36": Workload(
+        name="mix_gdn_b512h36", batch=512, heads=36, tokens=4096, window=16,
+        num_comp=4, bits=8, decay_kind="gdn", smoothing=True, seed=4),
+    "mix_kda_b512h12": Workload(
+        name="mix_kda_b512h12", batch=512, heads=12, tokens=4096, window=16,
+        num_comp=4, bits=8, decay_kind="kda", smoothing=True,
+        slow_channels=8, seed=1004),
 }
 
 
