@@ -79,10 +79,21 @@ template <int D>
 using TileReg = float2[FT<D>::IP][FT<D>::TJ];
 
 // scratch: dred [WC][D] f64 | dredc [WR][D] f64 | red [WC][D] | redc [WR][D]
-// | line [2][D] | pick [16]; then D*D bytes of unpacked codes (packed formats)
+// | taken lines [kMaxComp][D] | pick [16]; then D*D bytes of unpacked codes
+// (packed formats)
 template <int D>
 __host__ __device__ constexpr uint32_t compress_scratch_bytes() {
-    return align_up(8u * (FT<D>::WC + FT<D>::WR) * D + 4u * ((FT<D>::WC + FT<D>::WR + 2u) * D + 16u), 128u);
+    return align_up(8u * (FT<D>::WC + FT<D>::WR) * D + 4u * ((FT<D>::WC + FT<D>::WR + kMaxComp) * D + 16u),
+                    128u);
+}
+
+// (energy bits, key) of the better of two candidates: larger energy, then
+// the lower key; `a` holds the lower key
+__device__ __forceinline__ void pick_better(long long &ea, uint32_t &ka, long long eb, uint32_t kb) {
+    if (eb > ea) {
+        ea = eb;
+        ka = kb;
+    }
 }
 
 template <int D, int BITS>
@@ -347,8 +358,8 @@ __device__ int compress_tile(TileReg<D> &P, const Flags &F, const Layout &L, uin
     double *dredc = dred + WC * D;                        // [WR][D]
     float *red = reinterpret_cast<float *>(dredc + WR * D);
     float *redc = red + WC * D;
-    float *line = redc + WR * D;  // [2][D]
-    uint32_t *pick = reinterpret_cast<uint32_t *>(line + 2 * D);
+    float *line = redc + WR * D;  // [kMaxComp][D]
+    uint32_t *pick = reinterpret_cast<uint32_t *>(line + kMaxComp * D);
     int8_t *codes8 = reinterpret_cast<int8_t *>(scratch + compress_scratch_bytes<D>());
     float *cvec_out = reinterpret_cast<float *>(blob + L.cvec_off);
 
@@ -392,19 +403,31 @@ __device__ int compress_tile(TileReg<D> &P, const Flags &F, const Layout &L, uin
     int ncomp = 0;
     for (int cc = 0; cc < F.num_comp; ++cc) {
         // Non-negative doubles order like their bit patterns (negative
-        // rounding residue never wins against 0).  Keys: rows 0..D-1, then
-        // columns D..2D-1; strict comparisons in key order keep the lower key.
-        long long bb = 0;
-        uint32_t key = 0xFFFFFFFFu;
+        // rounding residue is clamped to 0, and 0 never wins).  Keys: rows
+        // 0..D-1, then columns D..2D-1; a pairwise tree in key order whose
+        // strict comparisons keep the lower key on ties.
+        long long ev[2 * KE];
+        uint32_t kv[2 * KE];
 #pragma unroll
         for (int k = 0; k < KE; ++k) {
-            const long long e = __double_as_longlong(rE[k]);
-            if (e > bb) { bb = e; key = lane + 32 * k; }
+            ev[k] = __double_as_longlong(rE[k]);
+            kv[k] = lane + 32 * k;
+            ev[KE + k] = __double_as_longlong(cE[k]);
+            kv[KE + k] = D + lane + 32 * k;
         }
 #pragma unroll
-        for (int k = 0; k < KE; ++k) {
-            const long long e = __double_as_longlong(cE[k]);
-            if (e > bb) { bb = e; key = D + lane + 32 * k; }
+        for (int n = KE; n >= 1; n >>= 1)
+#pragma unroll
+            for (int i = 0; i < n; ++i) {
+                ev[i] = ev[2 * i];
+                kv[i] = kv[2 * i];
+                pick_better(ev[i], kv[i], ev[2 * i + 1], kv[2 * i + 1]);
+            }
+        long long bb = ev[0];
+        uint32_t key = kv[0];
+        if (bb <= 0) {
+            bb = 0;
+            key = 0xFFFFFFFFu;
         }
         const uint32_t hi = (uint32_t)((unsigned long long)bb >> 32), lo = (uint32_t)bb;
         const uint32_t mhi = __reduce_max_sync(0xFFFFFFFFu, hi);
@@ -414,8 +437,7 @@ __device__ int compress_tile(TileReg<D> &P, const Flags &F, const Layout &L, uin
         const bool col = key >= (uint32_t)D;
         const int idx = col ? (int)key - D : (int)key;
         if (tid == 0) pick[cc] = col ? (kCompCol | (uint32_t)idx) : (uint32_t)idx;
-        float *w = cvec_out + (size_t)cc * D;
-        float *ln = line + (cc & 1) * D;
+        float *ln = line + cc * D;  // copied to the blob after the last round
         if (col) {
             if (idx >= j0 && idx < j0 + TJ) {
 #pragma unroll
@@ -424,7 +446,6 @@ __device__ int compress_tile(TileReg<D> &P, const Flags &F, const Layout &L, uin
 #pragma unroll
                         for (int ip = 0; ip < IP; ip += 2) {
                             const float4 v = make_float4(P[ip][jj].x, P[ip][jj].y, P[ip + 1][jj].x, P[ip + 1][jj].y);
-                            *reinterpret_cast<float4 *>(w + i0 + 2 * ip) = v;
                             *reinterpret_cast<float4 *>(ln + i0 + 2 * ip) = v;
                             P[ip][jj] = f2(0.f, 0.f);
                             P[ip + 1][jj] = f2(0.f, 0.f);
@@ -438,7 +459,6 @@ __device__ int compress_tile(TileReg<D> &P, const Flags &F, const Layout &L, uin
 #pragma unroll
                     for (int jj = 0; jj < TJ; jj += 4) {
                         const float4 v = make_float4(P[ip][jj].x, P[ip][jj + 1].x, P[ip][jj + 2].x, P[ip][jj + 3].x);
-                        *reinterpret_cast<float4 *>(w + j0 + jj) = v;
                         *reinterpret_cast<float4 *>(ln + j0 + jj) = v;
                     }
 #pragma unroll
@@ -448,7 +468,6 @@ __device__ int compress_tile(TileReg<D> &P, const Flags &F, const Layout &L, uin
 #pragma unroll
                     for (int jj = 0; jj < TJ; jj += 4) {
                         const float4 v = make_float4(P[ip][jj].y, P[ip][jj + 1].y, P[ip][jj + 2].y, P[ip][jj + 3].y);
-                        *reinterpret_cast<float4 *>(w + j0 + jj) = v;
                         *reinterpret_cast<float4 *>(ln + j0 + jj) = v;
                     }
 #pragma unroll
@@ -473,8 +492,8 @@ __device__ int compress_tile(TileReg<D> &P, const Flags &F, const Layout &L, uin
         }
         ++ncomp;
     }
-    for (int cc = ncomp; cc < F.num_comp; ++cc)
-        for (int x = tid; x < D; x += kGroup) cvec_out[(size_t)cc * D + x] = 0.f;
+    // the taken lines (every round ended with a barrier), then zeros
+    for (int x = tid; x < F.num_comp * D; x += kGroup) cvec_out[x] = x < ncomp * D ? line[x] : 0.f;
 
     // ---- residual smoothing: one power of two per key row
     const float sm_lo = F.f16_scale ? 0x1p-14f : 0x1p-126f;
@@ -562,15 +581,20 @@ __device__ int compress_tile(TileReg<D> &P, const Flags &F, const Layout &L, uin
     int8_t *dst8 = BITS == 8 ? reinterpret_cast<int8_t *>(blob + L.codes_off) : codes8;
     const uint32_t dst_row = BITS == 8 ? L.row_bytes : (uint32_t)D;
     const float min_fast = F.f16_scale ? 0x1p-14f : 0x1p-100f;
+    constexpr int NW = TI / 4;  // code words per column of the tile
+    float inv[TJ];
+#pragma unroll
+    for (int jj = 0; jj < TJ; ++jj) inv[jj] = __frcp_rn(qsj[jj]);
+    uint32_t cw[TJ][NW];
+    unsigned slowm = 0u;  // columns that need the division
 #pragma unroll
     for (int jj = 0; jj < TJ; ++jj) {
         const float s = qsj[jj];
-        const float inv = __frcp_rn(s);
         uint32_t nb[TI];
         float dmax = 0.f;
 #pragma unroll
         for (int ip = 0; ip < IP; ++ip) {
-            const float2 tq = __fmul2_rn(P[ip][jj], f2(inv, inv));
+            const float2 tq = __fmul2_rn(P[ip][jj], f2(inv[jj], inv[jj]));
             const float2 nf = __fadd2_rn(tq, f2(12582912.0f, 12582912.0f));  // 1.5 * 2^23
             const float2 back = __fadd2_rn(nf, f2(-12582912.0f, -12582912.0f));
             const float2 d = __fadd2_rn(tq, f2(-back.x, -back.y));
@@ -578,10 +602,18 @@ __device__ int compress_tile(TileReg<D> &P, const Flags &F, const Layout &L, uin
             nb[2 * ip] = __float_as_uint(nf.x);
             nb[2 * ip + 1] = __float_as_uint(nf.y);
         }
-        if (s == 0.f) {
+        const bool zero = s == 0.f;
+        if (!zero && (!(s >= min_fast) || dmax > 0.49998f)) slowm |= 1u << jj;
 #pragma unroll
-            for (int ii = 0; ii < TI; ++ii) nb[ii] = 0u;
-        } else if (!(s >= min_fast) || dmax > 0.49998f) {
+        for (int w = 0; w < NW; ++w)
+            cw[jj][w] = zero ? 0u : pack4_low_bytes(nb[4 * w], nb[4 * w + 1], nb[4 * w + 2], nb[4 * w + 3]);
+    }
+    if (slowm) {
+#pragma unroll
+        for (int jj = 0; jj < TJ; ++jj) {
+            if (!((slowm >> jj) & 1u)) continue;
+            const float s = qsj[jj];
+            uint32_t nb[TI];
 #pragma unroll
             for (int ip = 0; ip < IP; ++ip) {
                 float a = __fdiv_rn(P[ip][jj].x, s), b = __fdiv_rn(P[ip][jj].y, s);
@@ -590,15 +622,16 @@ __device__ int compress_tile(TileReg<D> &P, const Flags &F, const Layout &L, uin
                 nb[2 * ip] = __float_as_uint(__fadd_rn(a, 12582912.0f));
                 nb[2 * ip + 1] = __float_as_uint(__fadd_rn(b, 12582912.0f));
             }
+#pragma unroll
+            for (int w = 0; w < NW; ++w)
+                cw[jj][w] = pack4_low_bytes(nb[4 * w], nb[4 * w + 1], nb[4 * w + 2], nb[4 * w + 3]);
         }
+    }
+#pragma unroll
+    for (int jj = 0; jj < TJ; ++jj) {
         int8_t *row = dst8 + (size_t)(j0 + jj) * dst_row + i0;
-        const uint32_t w0 = pack4_low_bytes(nb[0], nb[1], nb[2], nb[3]);
-        if constexpr (TI == 8) {
-            const uint32_t w1 = pack4_low_bytes(nb[4], nb[5], nb[6], nb[7]);
-            *reinterpret_cast<uint2 *>(row) = make_uint2(w0, w1);
-        } else {
-            *reinterpret_cast<uint32_t *>(row) = w0;
-        }
+        if constexpr (NW == 2) *reinterpret_cast<uint2 *>(row) = make_uint2(cw[jj][0], cw[jj][1]);
+        else *reinterpret_cast<uint32_t *>(row) = cw[jj][0];
     }
     if constexpr (BITS != 8) {
         gsync();
