@@ -537,15 +537,14 @@ def main_reference(args):
         _, _, used = oracle.run(p, *sample(nheads, x * nheads))
     dt = time.perf_counter() - t0
     value = args.steps * nheads * W / dt
-    args.layers = 1
-    desc = (f"per step: {nheads} heads x {W} tokens (one window incl. its flush) of "
-            f"{wl.name}, FP64 C oracle, OpenMP over heads")
+    desc = (f"per step: {nheads} heads x {W} tokens (one window incl. its flush) of one "
+            f"{wl.name} layer, FP64 C oracle, OpenMP over heads")
     print(json.dumps({
         "metric": "decode head-tokens/s and achieved HBM GB/s (% of B200 peak) vs FP32-state kernel",
         "value": value, "unit": "head-tokens/s", "n_gpus": world, "steps": args.steps,
         "warmup": args.warmup, "ms_per_step": dt / args.steps * 1e3, "higher_is_better": True,
         "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": "synthetic",
-        "config": config_of(wl, args, 1), "impl": "reference",
+        "config": config_of(wl, args, world), "impl": "reference",
         "cpu_baseline": {"value": value, "unit": "head-tokens/s", "cores": used, "kind": "oracle",
                          "sample": desc},
         "e2e": {"value": value, "unit": "head-tokens/s", "h2d_bytes_per_step": 0,
