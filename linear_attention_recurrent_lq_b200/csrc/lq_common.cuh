@@ -139,6 +139,13 @@ __device__ __forceinline__ void bulk_g2s(void *smem_dst, const void *gmem_src, u
         : "memory");
 }
 
+// Bulk prefetch of global memory into L2 (no shared memory, no completion
+// tracking, no effect on the data seen later: L2 stays coherent with any
+// writer).  Address 16-byte aligned, bytes % 16 == 0.
+__device__ __forceinline__ void bulk_prefetch_l2(const void *gmem, uint32_t bytes) {
+    asm volatile("cp.async.bulk.prefetch.L2.global [%0], %1;" ::"l"(gmem), "r"(bytes) : "memory");
+}
+
 // Programmatic dependent launch: a kernel launched with programmatic stream
 // serialization may start while the previous kernel on the stream finishes;
 // pdl_wait() blocks until that kernel has completed and its memory is

@@ -282,6 +282,12 @@ __global__ void __launch_bounds__(D + 64) decode_kernel(DecodeArgs A) {
         fence_mbar_init();
     }
     __syncthreads();
+    // While the previous kernel on the stream drains, start pulling this
+    // CTA's first two blobs (compact state and codes) into L2.  A prefetch
+    // changes no data, so it is safe whatever that kernel writes.
+    if (tid == 0)
+        for (int it = 0; it < 2 && it < n_mine; ++it)
+            bulk_prefetch_l2(A.state + ((size_t)blockIdx.x + (size_t)it * G) * L.blob, L.pairs_off);
     pdl_wait();
     pdl_trigger();
 

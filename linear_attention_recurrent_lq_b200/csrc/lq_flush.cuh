@@ -735,6 +735,11 @@ __global__ void __launch_bounds__(kGroup, 2) flush_kernel(FlushArgs A) {
     uint8_t *stages = scratch + group_smem_bytes<D, BITS>();
     auto blob_at = [&](int it) { return A.state + ((size_t)blockIdx.x + (size_t)it * G) * L.blob; };
 
+    // pull the first two blobs into L2 while the previous kernel drains (a
+    // prefetch changes no data)
+    if (tid == 0)
+        for (int it = 0; it < kFlushStages && it < n_mine; ++it)
+            bulk_prefetch_l2(blob_at(it), L.pairs_off + (uint32_t)F.window * L.pair_bytes);
     pdl_wait();
     pdl_trigger();
     if (tid == 0) {
