@@ -26,7 +26,8 @@ NONE = 0xFFFFFFFF
 
 class _Params(ctypes.Structure):
     _fields_ = [(n, ctypes.c_int32) for n in
-                ("dk", "dv", "window", "num_comp", "bits", "kda", "smoothing", "scale_f16")]
+                ("dk", "dv", "window", "num_comp", "bits", "kda", "smoothing", "scale_f16",
+                 "per_step")]
 
 
 @dataclass(frozen=True)
@@ -39,6 +40,7 @@ class Params:
     kda: bool = False
     smoothing: bool = True
     scale_f16: bool = False
+    per_step: bool = False  # naive baselines: bits 16 = BF16, bits 8 = FP8 E4M3 state
 
     @property
     def qmax(self) -> int:
@@ -50,7 +52,7 @@ class Params:
 
     def c(self) -> _Params:
         return _Params(self.dk, self.dv, self.window, self.num_comp, self.bits,
-                       int(self.kda), int(self.smoothing), int(self.scale_f16))
+                       int(self.kda), int(self.smoothing), int(self.scale_f16), int(self.per_step))
 
     @staticmethod
     def of(wl) -> "Params":
@@ -80,6 +82,11 @@ def bind(path: str):
                                       vp, vp, vp, vp, vp]
     L.lqo_round_f16.restype = ctypes.c_double
     L.lqo_round_f16.argtypes = [ctypes.c_double]
+    L.lqo_round_bf16.restype = ctypes.c_double
+    L.lqo_round_bf16.argtypes = [ctypes.c_double]
+    L.lqo_round_e4m3.restype = ctypes.c_double
+    L.lqo_round_e4m3.argtypes = [ctypes.c_double]
+    L.lqo_fp8_columns.argtypes = [ctypes.c_int, ctypes.c_int, vp, vp, vp]
     L.lqo_row_bytes.restype = ctypes.c_int
     L.lqo_row_bytes.argtypes = [ctypes.c_int, ctypes.c_int]
     L.lqo_pack_rows.argtypes = [ctypes.c_int, ctypes.c_int, ctypes.c_int, vp, vp]
@@ -212,6 +219,25 @@ def window_buffered(S_base, q, k, v, beta, a):
 
 def round_f16(x: float) -> float:
     return lib().lqo_round_f16(float(x))
+
+
+def round_bf16(x: float) -> float:
+    return lib().lqo_round_bf16(float(x))
+
+
+def round_e4m3(x: float) -> float:
+    return lib().lqo_round_e4m3(float(x))
+
+
+def fp8_columns(S32):
+    """Per-value-column FP8 E4M3 quantization of an FP32 state [dk, dv]:
+    (scale [dv] float32, code values [dk, dv] float32)."""
+    S32, sp = _c(S32, np.float32)
+    dk, dv = S32.shape
+    scale = np.zeros(dv, np.float32)
+    val = np.zeros((dk, dv), np.float32)
+    lib().lqo_fp8_columns(dk, dv, sp, scale.ctypes.data, val.ctypes.data)
+    return scale, val
 
 
 def row_bytes(bits: int, dk: int) -> int:

@@ -32,7 +32,10 @@
  *     or above its absolute maximum (1 for an all-zero row);
  *   - quantization is symmetric per value column of the smoothed residual,
  *     scale = fl32(absmax / Qmax) rounded to the storage dtype, codes =
- *     clamp(rint(fl32(R'/scale)), -Qmax, Qmax), ties to even.
+ *     clamp(rint(fl32(R'/scale)), -Qmax, Qmax), ties to even;
+ *   - the naive per-step baselines of the accuracy table (BF16, FP8) store the
+ *     whole FP32-rounded state after every token: BF16 entry by entry, FP8 as
+ *     E4M3 codes with one FP32 scale fl32(absmax / 448) per value column.
  */
 #include <math.h>
 #include <stdint.h>
@@ -51,6 +54,9 @@ typedef struct {
     int32_t kda;        /* 0: scalar decay per head, 1: per key channel */
     int32_t smoothing;  /* 0/1 */
     int32_t scale_f16;  /* 0: scales stored in f32, 1: in f16 */
+    int32_t per_step;   /* 1: the naive per-step baselines: a dense state stored
+                           after every token as BF16 (bits 16) or as FP8 E4M3
+                           codes with one FP32 scale per value column (bits 8) */
 } lqo_params;
 
 #define LQO_KIND_COL 0x80000000u
@@ -295,6 +301,80 @@ static void to_f32(int n, const double *x, float *y)
     for (int i = 0; i < n; ++i) y[i] = (float)x[i];
 }
 
+/* Rounding to a binary floating-point format with `sig` significant bits
+ * (the implicit bit included) and smallest normal 2^emin, below which values
+ * keep the fixed quantum 2^(emin - sig + 1); round to nearest, ties to even.
+ * Written from the formats' definitions; returns the rounded value exactly. */
+static double round_format(double x, int sig, int emin)
+{
+    if (x != x || x == 0.0) return x;
+    double ax = fabs(x);
+    int e;
+    frexp(ax, &e);              /* ax = f * 2^e, f in [0.5, 1) */
+    int ex = e - 1;             /* floor(log2(ax)) */
+    if (ex < emin) ex = emin;
+    double quantum = ldexp(1.0, ex - (sig - 1));
+    double r = nearbyint(ax / quantum) * quantum;   /* ax/quantum is exact */
+    return x < 0 ? -r : r;
+}
+
+/* bfloat16: 8 significant bits, the exponent range of binary32 (largest
+ * finite 0x1.FEp127; beyond it the rounding gives infinity). */
+double lqo_round_bf16(double x)
+{
+    double r = round_format(x, 8, -126);
+    if (fabs(r) > 0x1.FEp127) return x > 0 ? INFINITY : -INFINITY;
+    return r;
+}
+
+/* FP8 E4M3 (the "fn" variant: no infinities, largest finite 448):
+ * 4 significant bits, smallest normal 2^-6; magnitudes that round beyond 448
+ * saturate to 448 (the saturating conversion the state uses). */
+double lqo_round_e4m3(double x)
+{
+    double r = round_format(x, 4, -6);
+    if (r > 448.0) return 448.0;
+    if (r < -448.0) return -448.0;
+    return r;
+}
+
+/* Per-value-column FP8 quantization of an FP32 state (row-major, dk x dv):
+ * scale_j = fl32(max_i |S_ij| / 448), val_ij = e4m3(fl32(S_ij / scale_j))
+ * (ties to even, saturating); an all-zero column has scale 0 and values 0.
+ * The divisions are the correctly rounded FP32 quotients (a binary64 quotient
+ * of two floats rounded once more to binary32 is correctly rounded). */
+void lqo_fp8_columns(int dk, int dv, const float *S32, float *scale, float *val)
+{
+    for (int j = 0; j < dv; ++j) {
+        float m = 0.f;
+        for (int i = 0; i < dk; ++i) m = fmaxf(m, fabsf(S32[i * dv + j]));
+        const float sc = (float)((double)m / 448.0);
+        scale[j] = sc;
+        for (int i = 0; i < dk; ++i)
+            val[i * dv + j] = sc == 0.f ? 0.f
+                                        : (float)lqo_round_e4m3((double)(float)((double)S32[i * dv + j] / (double)sc));
+    }
+}
+
+/* The naive per-step baselines ([NEWS] accuracy table: BF16 and FP8 states):
+ * after every token the state is rounded to FP32 and stored in the narrow
+ * format, and the next token starts from the stored values.  BF16: each entry
+ * rounded to bfloat16.  FP8: per-value-column E4M3 codes, dequantized as
+ * fl32(code * scale).                                                      */
+static void per_step_store(const lqo_params *p, double *S, float *buf32, float *scale, float *val)
+{
+    const int n = p->dk * p->dv;
+    to_f32(n, S, buf32);
+    if (p->bits == 16) {
+        for (int x = 0; x < n; ++x) S[x] = lqo_round_bf16((double)buf32[x]);
+        return;
+    }
+    lqo_fp8_columns(p->dk, p->dv, buf32, scale, val);
+    for (int i = 0; i < p->dk; ++i)
+        for (int j = 0; j < p->dv; ++j)
+            S[i * p->dv + j] = (double)(float)((double)val[i * p->dv + j] * (double)scale[j]);
+}
+
 /* Compress then dequantize, in place: the state after a window boundary. */
 static void requantize(const lqo_params *p, double *S, float *buf32, int8_t *codes, float *qs,
                        float *sm, uint32_t *meta, float *vec)
@@ -312,6 +392,8 @@ static void requantize(const lqo_params *p, double *S, float *buf32, int8_t *cod
  * plain result is the dense recurrence restarted from the dequantized state at
  * every boundary, which is what this computes.  bits == 32: no quantization at
  * all (the FP32-state reference).  A partial final window stays unquantized.
+ * per_step: the naive baselines instead, the whole state stored in BF16 or
+ * FP8 after every token (per_step_store).
  *
  *   S0    [nh*dk*dv] float         q,k [T*nh*dk]   v [T*nh*dv]
  *   beta  [T*nh]     decay [T*nh] (GDN) or [T*nh*dk] (KDA)
@@ -344,8 +426,10 @@ int lqo_run(const lqo_params *p, int nh, int T, const float *S0, const float *q,
         double *vd = (double *)malloc(sizeof(double) * dv), *ad = (double *)malloc(sizeof(double) * dk);
         double *od = (double *)malloc(sizeof(double) * dv);
 
+        float *val = (float *)malloc(sizeof(float) * (size_t)dk * dv);
         for (int x = 0; x < dk * dv; ++x) S[x] = (double)S0[(size_t)h * dk * dv + x];
-        if (p->bits != 32) requantize(p, S, buf32, codes, qs, sm, meta, vec);
+        if (p->per_step) per_step_store(p, S, buf32, qs, val);
+        else if (p->bits != 32) requantize(p, S, buf32, codes, qs, sm, meta, vec);
         int in_window = 0;
         for (int t = 0; t < T; ++t) {
             size_t th = (size_t)t * nh + h;
@@ -354,13 +438,15 @@ int lqo_run(const lqo_params *p, int nh, int T, const float *S0, const float *q,
             for (int i = 0; i < dk; ++i) ad[i] = p->kda ? decay[th * dk + i] : decay[th];
             lqo_step(dk, dv, S, qd, kd, vd, (double)beta[th], ad, od, NULL);
             for (int j = 0; j < dv; ++j) o[th * dv + j] = od[j];
-            if (p->bits != 32 && ++in_window == p->window) {
+            if (p->per_step) {
+                per_step_store(p, S, buf32, qs, val);
+            } else if (p->bits != 32 && ++in_window == p->window) {
                 requantize(p, S, buf32, codes, qs, sm, meta, vec);
                 in_window = 0;
             }
         }
         if (S_end) memcpy(S_end + (size_t)h * dk * dv, S, sizeof(double) * (size_t)dk * dv);
-        free(S); free(buf32); free(codes); free(qs); free(sm); free(meta); free(vec);
+        free(S); free(buf32); free(codes); free(qs); free(sm); free(meta); free(vec); free(val);
         free(qd); free(kd); free(vd); free(ad); free(od);
     }
     return used;

@@ -48,6 +48,16 @@ MUTATIONS = {
         "unsigned hi = (((unsigned)(uint8_t)cg[12 + b] & 0x3F) >> (4 - 2 * q)) & 0x3;"),
     "f16 rounding truncates": ("double r = nearbyint(ax / quantum) * quantum;",
                                "double r = floor(ax / quantum) * quantum;"),
+    "bf16 keeps one bit too many": ("double r = round_format(x, 8, -126);",
+                                    "double r = round_format(x, 9, -126);"),
+    "e4m3 does not saturate": ("if (r > 448.0) return 448.0;", "if (r > 480.0) return 448.0;"),
+    "fp8 scale for the wrong format maximum": ("const float sc = (float)((double)m / 448.0);",
+                                               "const float sc = (float)((double)m / 240.0);"),
+    "fp8 scale per key row": ("for (int i = 0; i < dk; ++i) m = fmaxf(m, fabsf(S32[i * dv + j]));",
+                              "for (int i = 0; i < dk; ++i) m = fmaxf(m, fabsf(S32[j * dv + i]));"),
+    "per-step state not stored after the token": (
+        "                per_step_store(p, S, buf32, qs, val);\n            } else",
+        "                ;\n            } else"),
 }
 
 PIN_TESTS = [getattr(pins, n) for n in dir(pins) if n.startswith("test_")]

@@ -426,3 +426,99 @@ def test_compensators_and_smoothing_reduce_error(oracle_lib):
         graded, num_comp=1, smoothing=False)
     e = [_err_vs_fp32(wl, bits=b, num_comp=3, smoothing=True) for b in (8, 6, 4)]
     assert e[0] < e[1] < e[2], e
+
+
+# --------------------------------------------------------------------------
+# the naive per-step baselines of the accuracy table (BF16 and FP8 states)
+
+def test_bf16_rounding_matches_torch(oracle_lib):
+    """bfloat16 rounding (ties to even, subnormals included) against
+    PyTorch's float32 -> bfloat16 conversion."""
+    torch = pytest.importorskip("torch")
+    rng = np.random.default_rng(7)
+    mags = 10.0 ** rng.uniform(-44, 37, 20000)
+    x = np.concatenate([rng.standard_normal(20000) * mags,
+                        [1 + 2.0 ** -8, 1 + 3 * 2.0 ** -9, -(1 + 2.0 ** -8), 1.5 * 2.0 ** -126,
+                         2.0 ** -133, 3 * 2.0 ** -134, 0.0]]).astype(np.float32)
+    ref = torch.from_numpy(x).to(torch.bfloat16).float().numpy()
+    got = np.array([oracle_lib.round_bf16(float(v)) for v in x], np.float32)
+    np.testing.assert_array_equal(got, ref)
+
+
+def test_e4m3_rounding_matches_torch_and_saturates(oracle_lib):
+    """FP8 E4M3 rounding against PyTorch's float32 -> float8_e4m3fn
+    conversion inside the finite range, and saturation to 448 beyond it (the
+    format's largest finite value)."""
+    torch = pytest.importorskip("torch")
+    rng = np.random.default_rng(8)
+    x = rng.standard_normal(20000) * 2.0 ** rng.integers(-12, 8, 20000)
+    x = np.concatenate([x[np.abs(x) <= 448], [2.0 ** -10, 3 * 2.0 ** -10, 1 + 2.0 ** -4, 1 + 3 * 2.0 ** -4,
+                                              248.0, -248.0, 448.0, 0.0]]).astype(np.float32)
+    ref = torch.from_numpy(x).to(torch.float8_e4m3fn).float().numpy()
+    got = np.array([oracle_lib.round_e4m3(float(v)) for v in x], np.float32)
+    np.testing.assert_array_equal(got, ref)
+    for v, want in ((449.0, 448.0), (464.0, 448.0), (470.0, 448.0), (1e6, 448.0), (-1e6, -448.0)):
+        assert oracle_lib.round_e4m3(v) == want, v
+
+
+def test_fp8_column_quantization_by_hand(oracle_lib):
+    """Per-value-column FP8: scale = fl32(column max / 448), codes = E4M3 of
+    the FP32 quotient; an all-zero column has scale 0."""
+    S = np.zeros((4, 3), np.float32)
+    S[:, 0] = [1.0, -0.5, 0.25, 0.0]
+    S[:, 2] = [1344.0, 3.0, -1344.0, 1.0]
+    scale, val = oracle_lib.fp8_columns(S)
+    assert scale[0] == np.float32(1.0) / np.float32(448.0)
+    assert scale[1] == 0.0 and scale[2] == 3.0
+    np.testing.assert_array_equal(val[:, 0], [448.0, -224.0, 112.0, 0.0])
+    np.testing.assert_array_equal(val[:, 1], [0.0, 0.0, 0.0, 0.0])
+    # 1/3 lies between the E4M3 values 0.3125 and 0.34375 (spacing 1/32 in [1/4, 1/2))
+    np.testing.assert_array_equal(val[:, 2], [448.0, 1.0, -448.0, 0.34375])
+
+
+@pytest.mark.parametrize("bits", [16, 8])
+def test_per_step_store_keeps_representable_states(oracle_lib, bits):
+    """With beta = 0 and decay 1/2 every state of the run is 2^-t S0.  If S0
+    is exactly representable in the per-step format (BF16 values; for FP8,
+    E4M3 values times a power-of-two column scale whose column maximum is
+    448 times that scale), storing it after every token changes nothing, and
+    the outputs equal those of the unquantized state exactly."""
+    rng = np.random.default_rng(9)
+    dk = dv = 16
+    grid = np.array([oracle_lib.round_e4m3(v) for v in rng.uniform(-448, 448, dk * dv)]).reshape(dk, dv)
+    if bits == 16:
+        S0 = np.array([oracle_lib.round_bf16(v) for v in rng.normal(0, 1, dk * dv)]).reshape(dk, dv)
+    else:
+        grid[0, :] = 448.0
+        S0 = grid * 2.0 ** -rng.integers(3, 9, dv)[None, :]
+    T = 8
+    q = np.stack([_unit(rng, dk) for _ in range(T)])[:, None]
+    k = np.stack([_unit(rng, dk) for _ in range(T)])[:, None]
+    v = rng.normal(size=(T, 1, dv))
+    beta = np.zeros((T, 1))
+    decay = np.full((T, 1), 0.5)
+    base = dict(dk=dk, dv=dv, window=1, num_comp=0, smoothing=False)
+    o_ref, S_ref, _ = oracle_lib.run(oracle_lib.Params(**base, bits=32), S0[None], q, k, v, beta, decay)
+    o, S, _ = oracle_lib.run(oracle_lib.Params(**base, bits=bits, per_step=True), S0[None], q, k, v, beta,
+                             decay)
+    np.testing.assert_array_equal(o, o_ref)
+    np.testing.assert_array_equal(S, S_ref)
+
+
+def test_naive_per_step_baselines_lose_more_than_leapquant(oracle_lib):
+    """Accuracy table of the news post: at the same 8 bits, states stored
+    naively after every token (FP8 E4M3, or INT8 without compensators and
+    smoothing) drift much further from the FP32 state than LeapQuant's
+    windowed INT8; BF16, with more mantissa bits than E4M3, drifts less than
+    FP8, and still more than LeapQuant INT8."""
+    from linear_attention_recurrent_lq_b200 import inputs
+    wl = inputs.WORKLOADS["gdn_int8_b1h1"].replace(tokens=96)
+    e_lq = _err_vs_fp32(wl, window=16, num_comp=2, smoothing=True)
+    e_int8 = _err_vs_fp32(wl, window=1, num_comp=0, smoothing=False)
+    e_fp8 = _err_vs_fp32(wl, bits=8, per_step=True)
+    e_bf16 = _err_vs_fp32(wl, bits=16, per_step=True)
+    assert e_lq < 0.5 * e_int8, (e_lq, e_int8)
+    assert e_lq < 0.5 * e_fp8, (e_lq, e_fp8)
+    assert e_bf16 < e_fp8, (e_bf16, e_fp8)
+    # the table's headline: 8-bit LeapQuant also beats the per-step BF16 state
+    assert e_lq < e_bf16, (e_lq, e_bf16)
