@@ -50,6 +50,8 @@ def parse_args():
     ap.add_argument("--e2e-steps", type=int, default=0, help="0: steps/10")
     ap.add_argument("--no-e2e", action="store_true")
     ap.add_argument("--no-fp32", action="store_true")
+    ap.add_argument("--no-baselines", action="store_true",
+                    help="skip the naive per-step BF16 / FP8 / INT8 states")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--cpu-seconds", type=float, default=10.0)
     return ap.parse_args()
@@ -88,6 +90,15 @@ def flush_bytes(wl):
     compact = f["qs"] + f["sm"] + f["cvec"] + f["codes"]
     return (f["hdr"] + f["meta"] + compact + wl.window * f["pair"] + f["g"]) + \
            (compact + f["meta"] + 16 + f["g"])
+
+
+def per_step_bytes(wl, fmt):
+    """Per-step baseline per head-token: read and write the stored state
+    (BF16 entries, or FP8 codes plus f32 column scales), read the inputs,
+    write the output."""
+    f = field_bytes(wl)
+    state = 2 * wl.dk * wl.dv if fmt == "bf16" else wl.dk * wl.dv + 4 * wl.dv
+    return 2 * state + f["inputs"] + f["out"]
 
 
 def fp32_bytes(wl):
@@ -220,10 +231,11 @@ def whole_job_rate(units_per_rank, world, ms):
 class Arm:
     """L layer-states of one workload on this GPU, with captured graphs."""
 
-    def __init__(self, wl, layers_data, bits, torch, B):
+    def __init__(self, wl, layers_data, bits, torch, B, per_step=False):
         self.wl, self.torch, self.B = wl, torch, B
-        self.cfg = B.config_for(wl, bits=bits)
+        self.cfg = B.config_for(wl, bits=bits, per_step=per_step)
         self.bits = bits
+        self.has_flush = bits != 32 and not per_step
         self.L = len(layers_data)
         self.states, self.inp, self.out = [], [], []
         for ld in layers_data:
@@ -244,7 +256,7 @@ class Arm:
                                     self.out[l][t])
 
     def flush_all(self):
-        if self.bits == 32:
+        if not self.has_flush:
             return
         for l in range(self.L):
             self.states[l].flush()
@@ -260,18 +272,18 @@ class Arm:
         self.g_dec, self.g_fl = torch.cuda.CUDAGraph(), torch.cuda.CUDAGraph()
         with torch.cuda.graph(self.g_dec, stream=s):
             self.decode_all()
-        if self.bits != 32:
+        if self.has_flush:
             with torch.cuda.graph(self.g_fl, stream=s):
                 self.flush_all()
         torch.cuda.synchronize()
 
     def step(self):
         self.g_dec.replay()
-        if self.bits != 32:
+        if self.has_flush:
             self.g_fl.replay()
 
     def launches_per_step(self):
-        return self.wl.window * self.L + (self.L if self.bits != 32 else 0)
+        return self.wl.window * self.L + (self.L if self.has_flush else 0)
 
 
 def time_arm(arm, steps, warmup, torch, dist, world):
@@ -292,7 +304,7 @@ def time_arm(arm, steps, warmup, torch, dist, world):
         a.record()
         arm.g_dec.replay()
         b.record()
-        if arm.bits != 32:
+        if arm.has_flush:
             arm.g_fl.replay()
         c.record()
     end.record()
@@ -475,6 +487,31 @@ def main_ours(args):
         line["vs_fp32_state_kernel"] = value / v32
         del arm32
         torch.cuda.empty_cache()
+
+    # ---- the naive per-step baselines of the accuracy table on the same inputs:
+    # BF16 and FP8 E4M3 states stored after every token, and INT8 per step
+    # (LeapQuant's layout with W = 1, no compensators, no smoothing)
+    if not args.no_baselines:
+        base = {}
+        kb = args.fp32_steps or max(4, args.steps // 4)
+        wl1 = wl.replace(window=1, num_comp=0, smoothing=False)
+        for name, arm_wl, bits, per_step, bytes_tok in (
+                ("bf16", wl, 16, True, per_step_bytes(wl, "bf16")),
+                ("fp8_e4m3", wl, 8, True, per_step_bytes(wl, "fp8")),
+                ("int8", wl1, 8, False, decode_bytes(wl1, 0) + flush_bytes(wl1))):
+            armb = Arm(arm_wl, layers, bits, torch, B, per_step=per_step)
+            armb.capture()
+            ksb = kb * (wl.window // arm_wl.window)
+            tb, db, _ = time_arm(armb, ksb, max(3, args.warmup // 2), torch, dist, world)
+            units = ksb * arm_wl.window * L * nh
+            vb = whole_job_rate(units, world, tb)
+            ab = nh * bytes_tok * ksb * arm_wl.window * L / (tb / 1e3) / 1e9
+            base[name] = {"value": vb, "unit": "head-tokens/s", "steps": ksb,
+                          "bytes_per_head_token": bytes_tok, "achieved_gbs": ab, "frac": ab / hbm,
+                          "leapquant_speedup": value / vb}
+            del armb
+            torch.cuda.empty_cache()
+        line["per_step_baselines"] = base
 
     # ---- end to end through the public calls with host buffers
     if not args.no_e2e:

@@ -67,6 +67,20 @@
  * The blob holds no pointers: copying it snapshots or restores a state (a
  * prefix-cache entry after lq_window_flush is the prefix up to `pairs`).
  * bits = 32 (the FP32-state reference): header, then f32 S[dk][dv] at 128.
+ *
+ * Naive per-step baselines (per_step = 1), the comparison points of the
+ * accuracy table of the news post: the dense state is stored in a narrow
+ * format after every token, with no window, compensators or smoothing.
+ *    bits 16 (BF16): header, then bf16 S[dk][dv] at 128; each entry is the
+ *         bfloat16 rounding (ties to even) of its FP32 value.
+ *    bits 8 (FP8 E4M3): header, then f32 scale[dv] at 128, then at
+ *         128 + align128(4 dv) uint8 codes[dk][dv], row = key channel; for
+ *         value column j, scale_j = fl32(max_i |S_ij| / 448) and code_ij =
+ *         E4M3(fl32(S_ij / scale_j)), ties to even, saturating at 448 (an
+ *         all-zero column has scale 0 and codes 0); the value is
+ *         fl32(E4M3 value * scale_j).
+ * Per-step INT8 without compensators or smoothing is the LeapQuant layout
+ * with window = 1, num_comp = 0, smoothing = 0.
  */
 #ifndef LEAPQUANT_H
 #define LEAPQUANT_H
@@ -116,6 +130,10 @@ typedef struct lq_config {
     int32_t scale_dtype; /* 0: qs/sm stored as f32; 1: as f16                 */
     int32_t smoothing;   /* 1: per-key-row residual smoothing; 0: sm = 1      */
     int32_t in_dtype;    /* q, k, v element type: 0 f32, 1 bf16               */
+    int32_t per_step;    /* 0: LeapQuant (bits 8/6/4) or FP32 (bits 32);
+                            1: naive per-step state, bits 16 = BF16 or
+                            bits 8 = FP8 E4M3 (window, num_comp, smoothing and
+                            scale_dtype are then not used)                    */
 } lq_config;
 
 /* LQ_OK if the configuration is valid and built, else why not.  Host only. */
@@ -129,7 +147,8 @@ LQ_API size_t lq_state_bytes(const lq_config *cfg);
  *   state [N*H blobs]            out, overwritten entirely (header reset)
  *   S0    [N, H, dk, dv] f32     in, row = key channel
  * Runs the window-boundary compression (compensator extraction, smoothing,
- * quantization) on S0; bits = 32 copies S0.  Source: the prefill state enters
+ * quantization) on S0; bits = 32 copies S0; per_step rounds S0 to its
+ * format.  Source: the prefill state enters
  * the quantized cache; per-window paragraph of the news post. */
 LQ_API lq_status lq_state_init(const lq_config *cfg, void *state, const float *S0, lq_stream_t stream);
 
@@ -154,7 +173,7 @@ LQ_API lq_status lq_decode_step(const lq_config *cfg, void *state, const void *q
  * requantize, and reset count = 0, g = 1 (news post: per-window, Compensator
  * Tokens and residual smoothing paragraphs).  A (slot, head) with an empty
  * window (count = 0) is left as is.  May be called on a partial window
- * (sequence end, prefix-cache snapshot).  bits = 32: no-op. */
+ * (sequence end, prefix-cache snapshot).  bits = 32 and per_step: no-op. */
 LQ_API lq_status lq_window_flush(const lq_config *cfg, void *state, lq_stream_t stream);
 
 /* Write the dense FP32 state each blob stands for, pending pairs included:

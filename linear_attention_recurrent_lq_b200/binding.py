@@ -31,24 +31,28 @@ class LQError(RuntimeError):
 class lq_config(ctypes.Structure):
     _fields_ = [(n, ctypes.c_int32) for n in (
         "num_slots", "num_heads", "dk", "dv", "window", "num_comp", "bits", "decay_kind",
-        "scale_dtype", "smoothing", "in_dtype")]
+        "scale_dtype", "smoothing", "in_dtype", "per_step")]
 
     def __repr__(self):
         return "lq_config(" + ", ".join(f"{n}={getattr(self, n)}" for n, _ in self._fields_) + ")"
 
 
 def make_config(num_slots, num_heads, dk=128, dv=128, window=16, num_comp=4, bits=8,
-                decay_kind="gdn", scale_dtype="f32", smoothing=True, in_dtype="bf16") -> lq_config:
+                decay_kind="gdn", scale_dtype="f32", smoothing=True, in_dtype="bf16",
+                per_step=False) -> lq_config:
+    """per_step=True selects the naive per-step baselines: bits 16 = BF16
+    state, bits 8 = FP8 E4M3 state (window, num_comp, smoothing unused)."""
     return lq_config(int(num_slots), int(num_heads), int(dk), int(dv), int(window), int(num_comp),
                      int(bits), 1 if decay_kind == "kda" else 0, 1 if scale_dtype == "f16" else 0,
-                     int(bool(smoothing)), 1 if in_dtype == "bf16" else 0)
+                     int(bool(smoothing)), 1 if in_dtype == "bf16" else 0, int(bool(per_step)))
 
 
-def config_for(wl, bits: int | None = None) -> lq_config:
-    """The lq_config of a generator Workload (optionally another bit width)."""
+def config_for(wl, bits: int | None = None, per_step: bool = False) -> lq_config:
+    """The lq_config of a generator Workload (optionally another bit width, or
+    one of the per-step baselines)."""
     return make_config(wl.batch, wl.heads, wl.dk, wl.dv, wl.window, wl.num_comp,
                        wl.bits if bits is None else bits, wl.decay_kind, wl.scale_dtype,
-                       wl.smoothing, wl.in_dtype)
+                       wl.smoothing, wl.in_dtype, per_step)
 
 
 def _load():

@@ -12,6 +12,7 @@
 #include "lq_decode.cuh"
 #include "lq_flush.cuh"
 #include "lq_fp32.cuh"
+#include "lq_perstep.cuh"
 
 using namespace lq;
 
@@ -24,8 +25,11 @@ lq_status check_config(const lq_config *c) {
     if (c->num_slots <= 0 || c->num_heads <= 0 || c->dk <= 0 || c->dv <= 0 || c->window <= 0 ||
         c->num_comp < 0)
         return LQ_ERR_INVALID_ARG;
-    if (c->bits != 4 && c->bits != 6 && c->bits != 8 && c->bits != 32) return LQ_ERR_INVALID_ARG;
-    if ((c->decay_kind | c->scale_dtype | c->smoothing | c->in_dtype) & ~1) return LQ_ERR_INVALID_ARG;
+    if ((c->decay_kind | c->scale_dtype | c->smoothing | c->in_dtype | c->per_step) & ~1)
+        return LQ_ERR_INVALID_ARG;
+    if (c->per_step ? (c->bits != 8 && c->bits != 16)
+                    : (c->bits != 4 && c->bits != 6 && c->bits != 8 && c->bits != 32))
+        return LQ_ERR_INVALID_ARG;
     if ((int64_t)c->num_slots * c->num_heads > 0x7FFFFFFF) return LQ_ERR_UNSUPPORTED;
     if (c->dk != c->dv || (c->dk != 64 && c->dk != 128)) return LQ_ERR_UNSUPPORTED;
     if (c->window > kMaxWindow || c->num_comp > kMaxComp) return LQ_ERR_UNSUPPORTED;
@@ -163,6 +167,22 @@ lq_status launch_fp32_decode(const lq_config &c, const Fp32Args &a, cudaStream_t
     return launched(launch_pdl(fp32_decode_kernel<D>, grid, kFp32Threads, 0u, s, a));
 }
 
+// The per-step baselines: one 128-thread CTA per (slot, head) and 64-column
+// block.  MODE 0 decode step, 1 store S0, 2 read back.
+template <int MODE>
+lq_status dispatch_perstep(const lq_config &c, const Fp32Args &a, cudaStream_t s) {
+    const int grid = a.num_heads * (c.dk / kPsCols);
+    cudaError_t e;
+    switch (c.dk * 100 + c.bits) {
+        case 12816: e = launch_pdl(perstep_kernel<128, 16, MODE>, grid, kFp32Threads, 0u, s, a); break;
+        case 12808: e = launch_pdl(perstep_kernel<128, 8, MODE>, grid, kFp32Threads, 0u, s, a); break;
+        case 6416: e = launch_pdl(perstep_kernel<64, 16, MODE>, grid, kFp32Threads, 0u, s, a); break;
+        case 6408: e = launch_pdl(perstep_kernel<64, 8, MODE>, grid, kFp32Threads, 0u, s, a); break;
+        default: return LQ_ERR_UNSUPPORTED;
+    }
+    return launched(e);
+}
+
 template <int MODE>
 lq_status launch_fp32_copy(const lq_config &c, const Fp32Args &a, cudaStream_t s) {
     const unsigned grid = (unsigned)(c.num_slots * c.num_heads);
@@ -192,6 +212,15 @@ lq_status lq_state_init(const lq_config *cfg, void *state, const float *S0, lq_s
     const lq_config &c = *cfg;
     const Layout L = make_layout(c);
     cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
+    if (c.per_step) {
+        Fp32Args a{};
+        a.state = static_cast<uint8_t *>(state);
+        a.S0 = S0;
+        a.L = L;
+        a.F = make_flags(c);
+        a.num_heads = c.num_slots * c.num_heads;
+        return dispatch_perstep<1>(c, a, s);
+    }
     if (c.bits == 32) {
         Fp32Args a{};
         a.state = static_cast<uint8_t *>(state);
@@ -215,6 +244,11 @@ lq_status lq_decode_step(const lq_config *cfg, void *state, const void *q, const
     const lq_config &c = *cfg;
     const Layout L = make_layout(c);
     cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
+    if (c.per_step) {
+        Fp32Args a{static_cast<uint8_t *>(state), nullptr, nullptr, L, make_flags(c), q, k, v,
+                   beta, decay, out, c.num_slots * c.num_heads};
+        return dispatch_perstep<0>(c, a, s);
+    }
     if (c.bits == 32) {
         Fp32Args a{static_cast<uint8_t *>(state), nullptr, nullptr, L, make_flags(c), q, k, v,
                    beta, decay, out, c.num_slots * c.num_heads};
@@ -239,7 +273,7 @@ lq_status lq_window_flush(const lq_config *cfg, void *state, lq_stream_t stream)
     if (!state) return LQ_ERR_INVALID_ARG;
     if (!aligned(state, 256)) return LQ_ERR_MISALIGNED;
     const lq_config &c = *cfg;
-    if (c.bits == 32) return LQ_OK;
+    if (c.bits == 32 || c.per_step) return LQ_OK;
     FlushArgs a{static_cast<uint8_t *>(state), nullptr, nullptr, make_layout(c), make_flags(c),
                 c.num_slots * c.num_heads};
     return dispatch_boundary<0>(c, a, reinterpret_cast<cudaStream_t>(stream));
@@ -254,6 +288,15 @@ lq_status lq_dequant_state(const lq_config *cfg, const void *state, float *S_out
     const Layout L = make_layout(c);
     cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
     uint8_t *st8 = const_cast<uint8_t *>(static_cast<const uint8_t *>(state));
+    if (c.per_step) {
+        Fp32Args a{};
+        a.state = st8;
+        a.S_out = S_out;
+        a.L = L;
+        a.F = make_flags(c);
+        a.num_heads = c.num_slots * c.num_heads;
+        return dispatch_perstep<2>(c, a, s);
+    }
     if (c.bits == 32) {
         Fp32Args a{};
         a.state = st8;

@@ -49,6 +49,14 @@ inline Layout make_layout(const lq_config &c) {
         L.blob = align_up(L.pairs_off, 256);
         return L;
     }
+    if (c.per_step) {
+        // BF16: S[dk][dv] bf16 at 128.  FP8: scale[dv] f32 at 128, codes[dk][dv] after it.
+        L.qs_off = L.sm_off = L.cvec_off = kHdrBytes;
+        L.codes_off = c.bits == 16 ? kHdrBytes : kHdrBytes + align_up(dv * 4, 128);
+        L.pairs_off = L.codes_off + dk * dv * (c.bits == 16 ? 2u : 1u);
+        L.blob = align_up(L.pairs_off, 256);
+        return L;
+    }
     L.scale_bytes = c.scale_dtype ? 2 : 4;
     L.row_bytes = dk * (uint32_t)c.bits / 8;
     L.pair_bytes = (dk + dv) * 4;

@@ -46,6 +46,12 @@ def test_state_bytes_follow_documented_layout(B):
                         assert L.blob % 256 == 0
     cfg = B.make_config(64, 32, bits=32)
     assert B.lq_state_bytes(cfg) == blob.layout(128, 128, 16, 4, 32, 0, 0).blob
+    # per-step baselines: header, then bf16 S; or f32 scales (128-aligned) and fp8 codes
+    for d in (64, 128):
+        bf16 = B.make_config(2, 3, d, d, bits=16, per_step=True)
+        fp8 = B.make_config(2, 3, d, d, bits=8, per_step=True)
+        assert B.lq_state_bytes(bf16) == (128 + 2 * d * d + 255) // 256 * 256
+        assert B.lq_state_bytes(fp8) == (128 + (4 * d + 127) // 128 * 128 + d * d + 255) // 256 * 256
 
 
 def test_headline_blob_size(B):
@@ -56,12 +62,20 @@ def test_headline_blob_size(B):
 @pytest.mark.parametrize("field,value,expect", [
     ("num_slots", 0, 1), ("num_heads", -1, 1), ("window", 0, 1), ("bits", 5, 1),
     ("decay_kind", 2, 1), ("scale_dtype", 3, 1), ("num_comp", -1, 1),
-    ("dk", 256, 2), ("dv", 64, 2), ("window", 65, 2), ("num_comp", 17, 2)])
+    ("dk", 256, 2), ("dv", 64, 2), ("window", 65, 2), ("num_comp", 17, 2), ("per_step", 2, 1),
+    ("bits", 16, 1)])
 def test_config_validation(B, field, value, expect):
     cfg = B.make_config(4, 4)
     setattr(cfg, field, value)
     assert B.lq_validate_config(cfg) == expect
     assert B.lib.lq_state_bytes(ctypes.byref(cfg)) == 0
+
+
+def test_per_step_formats_validate(B):
+    assert B.lq_validate_config(B.make_config(4, 4, bits=16, per_step=True)) == 0
+    assert B.lq_validate_config(B.make_config(4, 4, bits=8, per_step=True)) == 0
+    for bits in (4, 6, 32):
+        assert B.lq_validate_config(B.make_config(4, 4, bits=bits, per_step=True)) == 1
 
 
 def test_null_and_misaligned_pointers_rejected_before_launch(B):
