@@ -53,6 +53,8 @@ def parse_args():
     ap.add_argument("--no-baselines", action="store_true",
                     help="skip the naive per-step BF16 / FP8 / INT8 states")
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--no-slots", action="store_true",
+                    help="skip the serving path (decode and flush through a slot list)")
     ap.add_argument("--cpu-seconds", type=float, default=10.0)
     return ap.parse_args()
 
@@ -286,6 +288,42 @@ class Arm:
         return self.wl.window * self.L + (self.L if self.has_flush else 0)
 
 
+class SlotArm(Arm):
+    """The same layers served through a slot list: each layer's state buffer
+    holds 2x the running sequences, and the batch rows map to a seeded random
+    subset of those slots in shuffled order (continuous batching)."""
+
+    def __init__(self, wl, layers_data, torch, B, seed=12345):
+        import numpy as np
+        self.wl, self.torch, self.B = wl, torch, B
+        self.cfg = B.config_for(wl)
+        self.cfg.num_slots = 2 * wl.batch
+        self.bits, self.has_flush, self.L = wl.bits, True, len(layers_data)
+        rng = np.random.default_rng(seed)
+        pick = rng.permutation(2 * wl.batch)[:wl.batch]
+        self.slots = torch.from_numpy(pick.astype(np.int32)).cuda()
+        self.states, self.inp, self.out = [], [], []
+        for ld in layers_data:
+            st = B.LQState(self.cfg)
+            st.init_slots(self.slots, ld["S0"])
+            self.states.append(st)
+            self.inp.append(ld["dev"])
+            self.out.append(torch.empty((wl.window, wl.batch, wl.heads, wl.dv), dtype=torch.float32,
+                                        device="cuda"))
+        torch.cuda.synchronize()
+
+    def decode_all(self):
+        for t in range(self.wl.window):
+            for l in range(self.L):
+                x = self.inp[l]
+                self.states[l].step_slots(self.slots, x["q"][t], x["k"][t], x["v"][t], x["beta"][t],
+                                          x["decay"][t], self.out[l][t])
+
+    def flush_all(self):
+        for l in range(self.L):
+            self.states[l].flush_slots(self.slots)
+
+
 def time_arm(arm, steps, warmup, torch, dist, world):
     """Time `steps` window-steps; returns total ms (max over ranks) and the
     per-step decode / flush split from events recorded between the graphs."""
@@ -512,6 +550,25 @@ def main_ours(args):
             del armb
             torch.cuda.empty_cache()
         line["per_step_baselines"] = base
+
+    # ---- the serving path: the same work through a slot list
+    if not args.no_slots:
+        arms = SlotArm(wl, layers, torch, B)
+        arms.capture()
+        kss = args.fp32_steps or max(4, args.steps // 4)
+        ts, ds, fs = time_arm(arms, kss, max(3, args.warmup // 2), torch, dist, world)
+        status = max(st.check() for st in arms.states)
+        if status != 0:
+            raise RuntimeError(f"device status after the slot-list run: {B.STATUS_NAMES[status]}")
+        ds_ms = ds / (kss * W * L)
+        line["serving_slots"] = {
+            "value": whole_job_rate(kss * W * L * nh, world, ts), "unit": "head-tokens/s",
+            "steps": kss, "slots": f"{wl.batch} rows on a shuffled subset of {2 * wl.batch} slots",
+            "decode_avg_launch_us": ds_ms * 1e3,
+            "decode_frac": dec_bytes_per_launch / (ds_ms / 1e3) / 1e9 / hbm,
+            "flush_avg_launch_us": fs / (kss * L) * 1e3}
+        del arms
+        torch.cuda.empty_cache()
 
     # ---- end to end through the public calls with host buffers
     if not args.no_e2e:

@@ -188,6 +188,53 @@ LQ_API lq_status lq_dequant_state(const lq_config *cfg, const void *state, float
  * device pointer; the read uses one strided device-to-host copy. */
 LQ_API lq_status lq_check_status(const lq_config *cfg, const void *state, lq_stream_t stream);
 
+/* ---- Serving: a subset of the sequences through a slot list ----------
+ * A continuous-batching server keeps N sequence slots in one state buffer
+ * and decodes, at each step, only the sequences that are running.  The
+ * entry points below take those as a device list of slot indices:
+ *   slots  [n_active] int32, device, in: row n of the row-indexed tensors
+ *          belongs to the sequence in slot slots[n] (blobs slots[n]*H + h).
+ *          Entries must be distinct (two rows on one slot race: the result
+ *          is undefined, every access still stays inside the buffers).
+ * Every kernel bounds-checks each entry against [0, N): a row whose slot is
+ * out of range touches no blob; its output row (decode) is written as
+ * zeros.  n_active = 0 launches nothing and returns LQ_OK.  These three take
+ * the LeapQuant formats only (bits 8/6/4, per_step = 0), else
+ * LQ_ERR_UNSUPPORTED.  The list is read on the device when the kernel runs,
+ * so it may be written by earlier work on the same stream. */
+
+/* lq_state_init for the slots in `slots`:
+ *   S0 [n_active, H, dk, dv] f32, in (row n enters slot slots[n]).
+ * Status words of those slots are reset; other slots are not touched. */
+LQ_API lq_status lq_state_init_slots(const lq_config *cfg, void *state, const int32_t *slots,
+                                     int n_active, const float *S0, lq_stream_t stream);
+
+/* lq_decode_step for the slots in `slots`: q, k, v, beta, decay and out are
+ * laid out as for lq_decode_step with n_active rows in place of N.  The
+ * results of a row equal those lq_decode_step gives for that slot. */
+LQ_API lq_status lq_decode_step_slots(const lq_config *cfg, void *state, const int32_t *slots,
+                                      int n_active, const void *q, const void *k, const void *v,
+                                      const float *beta, const float *decay, float *out,
+                                      lq_stream_t stream);
+
+/* lq_window_flush for the slots in `slots` (slots reach their window
+ * boundary at different steps when sequences join at different times). */
+LQ_API lq_status lq_window_flush_slots(const lq_config *cfg, void *state, const int32_t *slots,
+                                       int n_active, lq_stream_t stream);
+
+/* Copy whole sequences between two state buffers with the blob layout of
+ * `cfg` (its num_slots is not used; any format, per_step and bits = 32
+ * included): for i < n, the H blobs of slot src_slots[i] of `src` (which
+ * holds src_num_slots slots) go to slot dst_slots[i] of `dst` (dst_num_slots
+ * slots).  Both lists are device int32 arrays; a pair with either index out
+ * of range is skipped.  A prefix cache snapshots a flushed sequence into a
+ * pool with it and restores it into a serving slot; the bytes are copied
+ * as they are, so a restored sequence continues bit for bit.  Source and
+ * destination blobs must not overlap. */
+LQ_API lq_status lq_copy_slots(const lq_config *cfg, void *dst, int dst_num_slots,
+                               const int32_t *dst_slots, const void *src, int src_num_slots,
+                               const int32_t *src_slots, int n, lq_stream_t stream);
+
 /* Static text for a status code. */
 LQ_API const char *lq_status_string(lq_status s);
 

@@ -19,7 +19,8 @@ STATUS_NAMES = {0: "LQ_OK", 1: "LQ_ERR_INVALID_ARG", 2: "LQ_ERR_UNSUPPORTED", 3:
                 4: "LQ_ERR_WINDOW_FULL", 5: "LQ_ERR_RANGE", 6: "LQ_ERR_MISALIGNED",
                 7: "LQ_ERR_TIMEOUT", 8: "LQ_ERR_CORRUPT"}
 ENTRY_POINTS = ("lq_validate_config", "lq_state_bytes", "lq_state_init", "lq_decode_step",
-                "lq_window_flush", "lq_dequant_state", "lq_check_status", "lq_status_string")
+                "lq_window_flush", "lq_dequant_state", "lq_check_status", "lq_state_init_slots",
+                "lq_decode_step_slots", "lq_window_flush_slots", "lq_copy_slots", "lq_status_string")
 
 
 class LQError(RuntimeError):
@@ -76,6 +77,15 @@ def _load():
     L.lq_dequant_state.restype = st
     L.lq_check_status.argtypes = [P, vp, vp]
     L.lq_check_status.restype = st
+    i32 = ctypes.c_int
+    L.lq_state_init_slots.argtypes = [P, vp, vp, i32, vp, vp]
+    L.lq_state_init_slots.restype = st
+    L.lq_decode_step_slots.argtypes = [P, vp, vp, i32, vp, vp, vp, vp, vp, vp, vp]
+    L.lq_decode_step_slots.restype = st
+    L.lq_window_flush_slots.argtypes = [P, vp, vp, i32, vp]
+    L.lq_window_flush_slots.restype = st
+    L.lq_copy_slots.argtypes = [P, vp, i32, vp, vp, i32, vp, i32, vp]
+    L.lq_copy_slots.restype = st
     L.lq_status_string.argtypes = [st]
     L.lq_status_string.restype = ctypes.c_char_p
     return L
@@ -150,6 +160,34 @@ def lq_check_status(cfg, state, stream=None) -> int:
     return lib.lq_check_status(ctypes.byref(cfg), _ptr(state), _stream(stream))
 
 
+def _n(slots) -> int:
+    return 0 if slots is None else int(slots.numel()) if hasattr(slots, "numel") else len(slots)
+
+
+def lq_state_init_slots(cfg, state, slots, S0, stream=None):
+    _check(lib.lq_state_init_slots(ctypes.byref(cfg), _ptr(state), _ptr(slots), _n(slots), _ptr(S0),
+                                   _stream(stream)), "lq_state_init_slots")
+
+
+def lq_decode_step_slots(cfg, state, slots, q, k, v, beta, decay, out, stream=None):
+    _check(lib.lq_decode_step_slots(ctypes.byref(cfg), _ptr(state), _ptr(slots), _n(slots), _ptr(q),
+                                    _ptr(k), _ptr(v), _ptr(beta), _ptr(decay), _ptr(out),
+                                    _stream(stream)), "lq_decode_step_slots")
+
+
+def lq_window_flush_slots(cfg, state, slots, stream=None):
+    _check(lib.lq_window_flush_slots(ctypes.byref(cfg), _ptr(state), _ptr(slots), _n(slots),
+                                     _stream(stream)), "lq_window_flush_slots")
+
+
+def lq_copy_slots(cfg, dst, dst_num_slots, dst_slots, src, src_num_slots, src_slots, stream=None):
+    if _n(dst_slots) != _n(src_slots):
+        raise ValueError("dst_slots and src_slots must have the same length")
+    _check(lib.lq_copy_slots(ctypes.byref(cfg), _ptr(dst), int(dst_num_slots), _ptr(dst_slots),
+                             _ptr(src), int(src_num_slots), _ptr(src_slots), _n(src_slots),
+                             _stream(stream)), "lq_copy_slots")
+
+
 class LQState:
     """N*H state blobs in one device buffer, with the library's calls bound."""
 
@@ -188,3 +226,13 @@ class LQState:
 
     def check(self, stream=None) -> int:
         return lq_check_status(self.cfg, self.buf, stream)
+
+    # slot lists: int32 device tensors of slot indices (one per active row)
+    def init_slots(self, slots, S0, stream=None):
+        lq_state_init_slots(self.cfg, self.buf, slots, S0, stream)
+
+    def step_slots(self, slots, q, k, v, beta, decay, out, stream=None):
+        lq_decode_step_slots(self.cfg, self.buf, slots, q, k, v, beta, decay, out, stream)
+
+    def flush_slots(self, slots, stream=None):
+        lq_window_flush_slots(self.cfg, self.buf, slots, stream)

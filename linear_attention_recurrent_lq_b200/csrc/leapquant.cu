@@ -119,7 +119,7 @@ int persistent_grid(K kernel, int threads, uint32_t smem, int work) {
 template <int D, int BITS>
 lq_status launch_decode(const lq_config &c, const DecodeArgs &a, cudaStream_t s) {
     const uint32_t smem = decode_smem_bytes(D, a.L, a.F);
-    auto k = decode_kernel<D, BITS>;
+    auto k = a.map.slots ? decode_kernel<D, BITS, true> : decode_kernel<D, BITS, false>;
     cudaError_t e = allow_smem(k, smem);
     if (e != cudaSuccess) return LQ_ERR_CUDA;
     const int threads = D + 64;
@@ -132,7 +132,7 @@ template <int D, int BITS, int MODE>
 lq_status launch_boundary(const lq_config &c, const FlushArgs &a, cudaStream_t s) {
     if (MODE == 0) {  // persistent flush
         const uint32_t smem = flush_smem_bytes(D, BITS, a.L, c.window);
-        auto k = flush_kernel<D, BITS>;
+        auto k = a.map.slots ? flush_kernel<D, BITS, true> : flush_kernel<D, BITS, false>;
         cudaError_t e = allow_smem(k, smem);
         if (e != cudaSuccess) return LQ_ERR_CUDA;
         const int threads = kGroup;
@@ -144,7 +144,7 @@ lq_status launch_boundary(const lq_config &c, const FlushArgs &a, cudaStream_t s
     auto k = boundary_kernel<D, BITS, MODE == 0 ? 1 : MODE>;
     cudaError_t e = allow_smem(k, smem);
     if (e != cudaSuccess) return LQ_ERR_CUDA;
-    k<<<(unsigned)(c.num_slots * c.num_heads), kGroup, smem, s>>>(a);
+    k<<<(unsigned)a.num_heads, kGroup, smem, s>>>(a);
     return launched(cudaSuccess);
 }
 
@@ -157,6 +157,18 @@ lq_status dispatch_boundary(const lq_config &c, const FlushArgs &a, cudaStream_t
         case 6408: return launch_boundary<64, 8, MODE>(c, a, s);
         case 6406: return launch_boundary<64, 6, MODE>(c, a, s);
         case 6404: return launch_boundary<64, 4, MODE>(c, a, s);
+        default: return LQ_ERR_UNSUPPORTED;
+    }
+}
+
+lq_status dispatch_decode(const lq_config &c, const DecodeArgs &a, cudaStream_t s) {
+    switch (c.dk * 100 + c.bits) {
+        case 12808: return launch_decode<128, 8>(c, a, s);
+        case 12806: return launch_decode<128, 6>(c, a, s);
+        case 12804: return launch_decode<128, 4>(c, a, s);
+        case 6408: return launch_decode<64, 8>(c, a, s);
+        case 6406: return launch_decode<64, 6>(c, a, s);
+        case 6404: return launch_decode<64, 4>(c, a, s);
         default: return LQ_ERR_UNSUPPORTED;
     }
 }
@@ -181,6 +193,31 @@ lq_status dispatch_perstep(const lq_config &c, const Fp32Args &a, cudaStream_t s
         default: return LQ_ERR_UNSUPPORTED;
     }
     return launched(e);
+}
+
+// Blob copy between two state buffers: CTA x moves blob x % H of pair x / H
+// with 16-byte loads and stores (a blob is a multiple of 256 bytes).  A pair
+// with either slot out of range is skipped.
+__global__ void __launch_bounds__(256) copy_slots_kernel(uint8_t *dst, int dst_slots_n, const int32_t *dst_slots,
+                                                         const uint8_t *src, int src_slots_n,
+                                                         const int32_t *src_slots, int heads, uint32_t blob) {
+    const int pair = blockIdx.x / heads, h = blockIdx.x % heads;
+    const int sd = __ldg(dst_slots + pair), ss = __ldg(src_slots + pair);
+    if (sd < 0 || sd >= dst_slots_n || ss < 0 || ss >= src_slots_n) return;
+    const uint4 *from = reinterpret_cast<const uint4 *>(src + ((size_t)ss * heads + h) * blob);
+    uint4 *to = reinterpret_cast<uint4 *>(dst + ((size_t)sd * heads + h) * blob);
+    for (uint32_t x = threadIdx.x; x < blob / 16u; x += 256u) to[x] = __ldg(from + x);
+}
+
+// Checks shared by the entry points that take a slot list.
+lq_status check_slots(const lq_config *cfg, const void *state, const int32_t *slots, int n_active) {
+    lq_status st = check_config(cfg);
+    if (st != LQ_OK) return st;
+    if (!state || n_active < 0 || (n_active > 0 && !slots)) return LQ_ERR_INVALID_ARG;
+    if (cfg->bits == 32 || cfg->per_step) return LQ_ERR_UNSUPPORTED;
+    if ((int64_t)n_active * cfg->num_heads > 0x7FFFFFFF) return LQ_ERR_UNSUPPORTED;
+    if (!aligned(state, 256) || !aligned(slots, 4)) return LQ_ERR_MISALIGNED;
+    return LQ_OK;
 }
 
 template <int MODE>
@@ -256,15 +293,7 @@ lq_status lq_decode_step(const lq_config *cfg, void *state, const void *q, const
     }
     DecodeArgs a{static_cast<uint8_t *>(state), L, make_flags(c), q, k, v, beta, decay, out,
                  c.num_slots * c.num_heads};
-    switch (c.dk * 100 + c.bits) {
-        case 12808: return launch_decode<128, 8>(c, a, s);
-        case 12806: return launch_decode<128, 6>(c, a, s);
-        case 12804: return launch_decode<128, 4>(c, a, s);
-        case 6408: return launch_decode<64, 8>(c, a, s);
-        case 6406: return launch_decode<64, 6>(c, a, s);
-        case 6404: return launch_decode<64, 4>(c, a, s);
-        default: return LQ_ERR_UNSUPPORTED;
-    }
+    return dispatch_decode(c, a, s);
 }
 
 lq_status lq_window_flush(const lq_config *cfg, void *state, lq_stream_t stream) {
@@ -330,6 +359,65 @@ lq_status lq_check_status(const lq_config *cfg, const void *state, lq_stream_t s
     if (any & LQ_DEV_TIMEOUT) return LQ_ERR_TIMEOUT;
     if (any & LQ_DEV_CORRUPT) return LQ_ERR_CORRUPT;
     return LQ_OK;
+}
+
+lq_status lq_state_init_slots(const lq_config *cfg, void *state, const int32_t *slots, int n_active,
+                              const float *S0, lq_stream_t stream) {
+    lq_status st = check_slots(cfg, state, slots, n_active);
+    if (st != LQ_OK) return st;
+    if (n_active > 0 && !S0) return LQ_ERR_INVALID_ARG;
+    if (!aligned(S0, 16)) return LQ_ERR_MISALIGNED;
+    if (n_active == 0) return LQ_OK;
+    const lq_config &c = *cfg;
+    FlushArgs a{static_cast<uint8_t *>(state), S0, nullptr, make_layout(c), make_flags(c),
+                n_active * c.num_heads, SlotMap{slots, c.num_heads, c.num_slots}};
+    return dispatch_boundary<1>(c, a, reinterpret_cast<cudaStream_t>(stream));
+}
+
+lq_status lq_decode_step_slots(const lq_config *cfg, void *state, const int32_t *slots, int n_active,
+                               const void *q, const void *k, const void *v, const float *beta,
+                               const float *decay, float *out, lq_stream_t stream) {
+    lq_status st = check_slots(cfg, state, slots, n_active);
+    if (st != LQ_OK) return st;
+    if (n_active > 0 && (!q || !k || !v || !beta || !decay || !out)) return LQ_ERR_INVALID_ARG;
+    if (!aligned(q, 16) || !aligned(k, 16) || !aligned(v, 16) || !aligned(beta, 4) ||
+        !aligned(decay, cfg->decay_kind ? 16 : 4) || !aligned(out, 4))
+        return LQ_ERR_MISALIGNED;
+    if (n_active == 0) return LQ_OK;
+    const lq_config &c = *cfg;
+    DecodeArgs a{static_cast<uint8_t *>(state), make_layout(c), make_flags(c), q, k, v, beta, decay, out,
+                 n_active * c.num_heads, SlotMap{slots, c.num_heads, c.num_slots}};
+    return dispatch_decode(c, a, reinterpret_cast<cudaStream_t>(stream));
+}
+
+lq_status lq_window_flush_slots(const lq_config *cfg, void *state, const int32_t *slots, int n_active,
+                                lq_stream_t stream) {
+    lq_status st = check_slots(cfg, state, slots, n_active);
+    if (st != LQ_OK) return st;
+    if (n_active == 0) return LQ_OK;
+    const lq_config &c = *cfg;
+    FlushArgs a{static_cast<uint8_t *>(state), nullptr, nullptr, make_layout(c), make_flags(c),
+                n_active * c.num_heads, SlotMap{slots, c.num_heads, c.num_slots}};
+    return dispatch_boundary<0>(c, a, reinterpret_cast<cudaStream_t>(stream));
+}
+
+lq_status lq_copy_slots(const lq_config *cfg, void *dst, int dst_num_slots, const int32_t *dst_slots,
+                        const void *src, int src_num_slots, const int32_t *src_slots, int n,
+                        lq_stream_t stream) {
+    lq_status st = check_config(cfg);
+    if (st != LQ_OK) return st;
+    if (!dst || !src || n < 0 || dst_num_slots <= 0 || src_num_slots <= 0 ||
+        (n > 0 && (!dst_slots || !src_slots)))
+        return LQ_ERR_INVALID_ARG;
+    if ((int64_t)n * cfg->num_heads > 0x7FFFFFFF) return LQ_ERR_UNSUPPORTED;
+    if (!aligned(dst, 256) || !aligned(src, 256) || !aligned(dst_slots, 4) || !aligned(src_slots, 4))
+        return LQ_ERR_MISALIGNED;
+    if (n == 0) return LQ_OK;
+    const uint32_t blob = make_layout(*cfg).blob;
+    copy_slots_kernel<<<(unsigned)(n * cfg->num_heads), 256, 0, reinterpret_cast<cudaStream_t>(stream)>>>(
+        static_cast<uint8_t *>(dst), dst_num_slots, dst_slots, static_cast<const uint8_t *>(src), src_num_slots,
+        src_slots, cfg->num_heads, blob);
+    return launched(cudaSuccess);
 }
 
 const char *lq_status_string(lq_status s) {

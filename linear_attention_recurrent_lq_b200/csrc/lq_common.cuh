@@ -72,6 +72,26 @@ inline Layout make_layout(const lq_config &c) {
     return L;
 }
 
+// Serving-side slot indirection.  Work item h (0 <= h < rows * H) is head
+// h % H of active row h / H, and its blob is that head of slot
+// slots[h / H] of the state buffer.  Without a slot array the work item is
+// the blob itself.  A slot index outside [0, num_slots) maps to -1: the work
+// item is skipped and no blob is touched.
+struct SlotMap {
+    const int32_t *slots;  // device, one per active row; null = identity
+    int heads;             // H
+    int num_slots;         // slots in the state buffer
+    // blob index of work item h (< 2^31, checked on the host), -1: none.
+    // The list is read through L2 only (never a possibly stale L1 line: a
+    // kernel may read it before its wait on the kernel that writes it).
+    __device__ __forceinline__ int blob(int h) const {
+        if (!slots) return h;
+        const int row = h / heads;
+        const int s = __ldcg(slots + row);
+        return (s >= 0 && s < num_slots) ? s * heads + (h - row * heads) : -1;
+    }
+};
+
 // Runtime switches that do not change a kernel's shape.
 struct Flags {
     int kda;        // per-key-channel decay

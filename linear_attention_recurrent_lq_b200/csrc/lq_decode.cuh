@@ -46,7 +46,8 @@ struct DecodeArgs {
     const void *q, *k, *v;
     const float *beta, *decay;
     float *out;
-    int num_heads;  // N * H
+    int num_heads;  // work items: N * H, or active rows * H with a slot map
+    SlotMap map;
 };
 
 constexpr int kDotSlots = kMaxWindow + kMaxComp;
@@ -84,12 +85,14 @@ constexpr int kInfoRun = 0, kInfoCount = 1, kInfoNrow = 2, kInfoNcol = 3, kInfoB
 template <int D>
 __host__ __device__ constexpr uint32_t decode_fixed_smem() {
     // barriers + control (128) | chunk sums float2 [D/16][D+1] | prep buffers [2]
-    // | dots float2 [kDotSlots] | producer batch [3*32]
-    return align_up(128u + 8u * (D / 16) * (D + 1) + 2u * PrepBuf<D>::bytes + 8u * kDotSlots + 3u * 32u * 4u,
+    // | dots float2 [kDotSlots] | producer batch [4*32]
+    return align_up(128u + 8u * (D / 16) * (D + 1) + 2u * PrepBuf<D>::bytes + 8u * kDotSlots + 4u * 32u * 4u,
                     128u);
 }
 
 constexpr int kDecodeStages = 2;
+// Prep-warp marker of a work item whose slot is out of range (never a status bit).
+constexpr uint32_t kSkipItem = 0xFFFFFFFFu;
 
 inline uint32_t decode_smem_bytes(int D, const Layout &L, const Flags &F) {
     const uint32_t fixed = D == 128 ? decode_fixed_smem<128>() : decode_fixed_smem<64>();
@@ -237,8 +240,10 @@ __device__ __forceinline__ float warp_sum(float x) {
     return x;
 }
 
-template <int D, int BITS>
-__global__ void __launch_bounds__(D + 64) decode_kernel(DecodeArgs A) {
+// SLOTS: work items reach their blobs through A.map (a separate instance, so
+// the plain path carries none of the lookups).
+template <int D, int BITS, bool SLOTS>
+__global__ void __launch_bounds__(D + 64, SLOTS ? 3 : 0) decode_kernel(DecodeArgs A) {
     constexpr int NC = D;            // consumer threads
     constexpr int LPR = D / 16;      // threads per row, one 16-key chunk each
     constexpr int RPT = D / 16;      // rows per thread (16 row groups)
@@ -258,6 +263,7 @@ __global__ void __launch_bounds__(D + 64) decode_kernel(DecodeArgs A) {
     const DecodeStage SG = decode_stage(L, D, F.window, F.bf16_in, F.kda);
     const int G = gridDim.x;
     const int n_mine = (A.num_heads - (int)blockIdx.x + G - 1) / G;
+    auto blob_of = [](const SlotMap &m, int h) { return SLOTS ? m.blob(h) : h; };
 
     extern __shared__ __align__(128) uint8_t smem[];
     uint64_t *full = reinterpret_cast<uint64_t *>(smem);  // [2] stage landed
@@ -270,6 +276,7 @@ __global__ void __launch_bounds__(D + 64) decode_kernel(DecodeArgs A) {
     uint32_t *s_cnt = reinterpret_cast<uint32_t *>(s_dot + kDotSlots);  // copy-warp batch [32]
     float *s_pbeta = reinterpret_cast<float *>(s_cnt + 32);
     float *s_palpha = s_pbeta + 32;
+    int *s_bidx = reinterpret_cast<int *>(s_palpha + 32);  // blob of each batch item, -1: none
     uint8_t *stages = smem + decode_fixed_smem<D>();
 
     if (tid == 0) {
@@ -284,10 +291,14 @@ __global__ void __launch_bounds__(D + 64) decode_kernel(DecodeArgs A) {
     __syncthreads();
     // While the previous kernel on the stream drains, start pulling this
     // CTA's first two blobs (compact state and codes) into L2.  A prefetch
-    // changes no data, so it is safe whatever that kernel writes.
+    // changes no data, so it is safe whatever that kernel writes.  (A slot
+    // list read here may still be changing: a stale entry, bounds-checked
+    // like any other, only wastes the prefetch.)
     if (tid == 0)
-        for (int it = 0; it < 2 && it < n_mine; ++it)
-            bulk_prefetch_l2(A.state + ((size_t)blockIdx.x + (size_t)it * G) * L.blob, L.pairs_off);
+        for (int it = 0; it < 2 && it < n_mine; ++it) {
+            const int b = blob_of(A.map, (int)blockIdx.x + it * G);
+            if (b >= 0) bulk_prefetch_l2(A.state + (size_t)b * L.blob, L.pairs_off);
+        }
     pdl_wait();
     pdl_trigger();
 
@@ -297,7 +308,9 @@ __global__ void __launch_bounds__(D + 64) decode_kernel(DecodeArgs A) {
             const int i = base + lane;
             if (i < n_mine) {
                 const size_t h = blockIdx.x + (size_t)i * G;
-                s_cnt[lane] = *reinterpret_cast<const uint32_t *>(A.state + h * L.blob + kHdrCount);
+                const int b = blob_of(A.map, (int)h);
+                s_bidx[lane] = (int)b;
+                s_cnt[lane] = b >= 0 ? *reinterpret_cast<const uint32_t *>(A.state + b * L.blob + kHdrCount) : 0u;
                 s_pbeta[lane] = A.beta[h];
                 s_palpha[lane] = F.kda ? 1.f : A.decay[h];
             }
@@ -311,13 +324,18 @@ __global__ void __launch_bounds__(D + 64) decode_kernel(DecodeArgs A) {
                         break;
                     }
                     const size_t h = blockIdx.x + (size_t)it * G;
-                    const uint8_t *blob = A.state + h * L.blob;
                     uint8_t *st = stages + (size_t)s * SG.bytes;
-                    const uint32_t c = s_cnt[x];
-                    const uint32_t cc = c < (uint32_t)F.window ? c : 0u;
                     float *aux = reinterpret_cast<float *>(st + SG.aux_off);
                     aux[0] = s_pbeta[x];
                     aux[1] = s_palpha[x];
+                    aux[2] = s_bidx[x] >= 0 ? 0.f : 1.f;  // 1: no blob for this work item
+                    if (s_bidx[x] < 0) {
+                        mbar_arrive_expect_tx(&full[s], 0u);  // nothing is staged
+                        continue;
+                    }
+                    const uint8_t *blob = A.state + (size_t)s_bidx[x] * L.blob;
+                    const uint32_t c = s_cnt[x];
+                    const uint32_t cc = c < (uint32_t)F.window ? c : 0u;
                     const uint32_t pb = cc * L.pair_bytes;
                     mbar_arrive_expect_tx(&full[s], L.codes_off + pb + 3 * SG.qkv_bytes +
                                                         (F.kda ? (uint32_t)D * 4u : 0u));
@@ -368,7 +386,10 @@ __global__ void __launch_bounds__(D + 64) decode_kernel(DecodeArgs A) {
                 newbits = LQ_DEV_CORRUPT;
             else if (hdr.y == 0 && hdr.x >= (uint32_t)F.window)
                 newbits = LQ_DEV_WINDOW_FULL;
+            // a work item without a blob: the stage holds stale bytes, skip it
+            if (reinterpret_cast<const float *>(st + SG.aux_off)[2] != 0.f) newbits = kSkipItem;
             bool run = hdr.y == 0 && newbits == 0;
+            if (newbits == kSkipItem) newbits = 0;
             float kq = 0.f;
             if (run) {
                 const int i0 = KPL * lane;
@@ -482,8 +503,9 @@ __global__ void __launch_bounds__(D + 64) decode_kernel(DecodeArgs A) {
     const uint8_t *code_base = A.state + L.codes_off + c * GB;
 
     Group<BITS> cg[RPT];
-    if (n_mine > 0) {
-        const uint8_t *cb = code_base + (size_t)blockIdx.x * L.blob;
+    const int b_first = n_mine > 0 ? blob_of(A.map, (int)blockIdx.x) : -1;
+    if (b_first >= 0) {
+        const uint8_t *cb = code_base + (size_t)b_first * L.blob;
 #pragma unroll
         for (int m = 0; m < RPT; ++m) load_group<BITS>(cg[m], cb + (size_t)(RPT * rg + m) * L.row_bytes);
     }
@@ -498,13 +520,20 @@ __global__ void __launch_bounds__(D + 64) decode_kernel(DecodeArgs A) {
         const uint8_t *st = stages + (size_t)s * SG.bytes;
         const uint8_t *pb = s_pb + (it & 1) * PB::bytes;
         const size_t h = blockIdx.x + (size_t)it * G;
-        uint8_t *blob = A.state + h * L.blob;
-        const bool has_next = it + 1 < n_mine;
+        const int bi = blob_of(A.map, (int)h);
+        uint8_t *blob = A.state + (bi >= 0 ? (size_t)bi : 0) * L.blob;
+        // codes of the next work item to load (through a slot map: if it has a blob)
+        bool has_next = it + 1 < n_mine;
         const uint8_t *next_codes = code_base + (h + G) * (size_t)L.blob;
+        if constexpr (SLOTS) {
+            const int bn = has_next ? A.map.blob((int)h + G) : -1;
+            has_next = bn >= 0;
+            next_codes = code_base + (size_t)(has_next ? bn : 0) * L.blob;
+        }
         if (!consumer_sync_and(mbar_wait_bounded(&pfull[s], ph), NC)) {
             // the data never arrived: record it on this blob and stop this CTA
             if (tid == 0) {
-                set_status(blob, LQ_DEV_TIMEOUT);
+                if (bi >= 0) set_status(blob, LQ_DEV_TIMEOUT);
                 *s_abort = 1u;
             }
             A.out[h * D + tid] = 0.f;

@@ -128,7 +128,8 @@ struct FlushArgs {
     float *S_out;     // dequant only
     Layout L;
     Flags F;
-    int num_heads;
+    int num_heads;  // work items: N * H, or active rows * H with a slot map
+    SlotMap map;
 };
 
 // barrier of the 256 threads that handle a blob
@@ -719,7 +720,8 @@ __device__ __forceinline__ uint32_t staged_bytes(const Layout &L, int window, ui
 // Thread 0 stages blob it + 2 as soon as every consumer has rebuilt blob it
 // (the barrier after the rebuild frees the stage); it reads that blob's
 // window count at the top of the iteration, so the load is long done.
-template <int D, int BITS>
+// SLOTS: work items reach their blobs through A.map (a separate instance).
+template <int D, int BITS, bool SLOTS>
 __global__ void __launch_bounds__(kGroup, 2) flush_kernel(FlushArgs A) {
     const int tid = threadIdx.x;
     const Layout L = A.L;
@@ -733,23 +735,30 @@ __global__ void __launch_bounds__(kGroup, 2) flush_kernel(FlushArgs A) {
     uint8_t *scratch = smem + 256;
     int8_t *codes8 = reinterpret_cast<int8_t *>(scratch + compress_scratch_bytes<D>());
     uint8_t *stages = scratch + group_smem_bytes<D, BITS>();
-    auto blob_at = [&](int it) { return A.state + ((size_t)blockIdx.x + (size_t)it * G) * L.blob; };
+    // the blob of work item it, or null when its slot is out of range
+    auto blob_at = [&](int it) -> uint8_t * {
+        const int b = SLOTS ? A.map.blob((int)blockIdx.x + it * G) : (int)blockIdx.x + it * G;
+        return b >= 0 ? A.state + (size_t)b * L.blob : nullptr;
+    };
 
     // pull the first two blobs into L2 while the previous kernel drains (a
-    // prefetch changes no data)
+    // prefetch changes no data; a slot list read here may still be changing:
+    // a stale entry, bounds-checked like any other, only wastes the prefetch)
     if (tid == 0)
-        for (int it = 0; it < kFlushStages && it < n_mine; ++it)
-            bulk_prefetch_l2(blob_at(it), L.pairs_off + (uint32_t)F.window * L.pair_bytes);
+        for (int it = 0; it < kFlushStages && it < n_mine; ++it) {
+            const uint8_t *b = blob_at(it);
+            if (b) bulk_prefetch_l2(b, L.pairs_off + (uint32_t)F.window * L.pair_bytes);
+        }
     pdl_wait();
     pdl_trigger();
     if (tid == 0) {
         for (int s = 0; s < kFlushStages; ++s) mbar_init(&full[s], 1);
         fence_mbar_init();
         for (int it = 0; it < kFlushStages && it < n_mine; ++it) {
-            const uint32_t c = *reinterpret_cast<const uint32_t *>(blob_at(it) + kHdrCount);
-            const uint32_t bytes = staged_bytes(L, F.window, c);
+            const uint8_t *b = blob_at(it);
+            const uint32_t bytes = b ? staged_bytes(L, F.window, *reinterpret_cast<const uint32_t *>(b + kHdrCount)) : 0u;
             mbar_arrive_expect_tx(&full[it], bytes);
-            bulk_g2s(stages + (size_t)it * SB, blob_at(it), bytes, &full[it]);
+            if (b) bulk_g2s(stages + (size_t)it * SB, b, bytes, &full[it]);
         }
     }
     __syncthreads();
@@ -759,11 +768,12 @@ __global__ void __launch_bounds__(kGroup, 2) flush_kernel(FlushArgs A) {
         const uint8_t *st = stages + (size_t)s * SB;
         uint8_t *blob = blob_at(it);
         const bool refill = tid == 0 && it + kFlushStages < n_mine;
+        uint8_t *blob_next = refill ? blob_at(it + kFlushStages) : nullptr;
         uint32_t c_next = 0;
-        if (refill) c_next = *reinterpret_cast<const volatile uint32_t *>(blob_at(it + kFlushStages) + kHdrCount);
+        if (blob_next) c_next = *reinterpret_cast<const volatile uint32_t *>(blob_next + kHdrCount);
         if (!gsync_and(mbar_wait_bounded(&full[s], (uint32_t)(it / kFlushStages) & 1u))) {
             if (tid == 0) {
-                set_status(blob, LQ_DEV_TIMEOUT);
+                if (blob) set_status(blob, LQ_DEV_TIMEOUT);
                 // let the copies still in flight land before the CTA leaves
                 for (int x = it; x < it + kFlushStages && x < n_mine; ++x)
                     mbar_wait_bounded(&full[x % kFlushStages], (uint32_t)(x / kFlushStages) & 1u);
@@ -772,8 +782,9 @@ __global__ void __launch_bounds__(kGroup, 2) flush_kernel(FlushArgs A) {
         }
         const StagedHeader H = parse_staged<D>(st, F);
         // flush only a valid blob with a non-empty window and no error flag
-        const bool run = H.ok && H.status == 0 && H.count > 0;
-        if (!H.ok && tid == 0) set_status(blob, LQ_DEV_CORRUPT);
+        // (a work item without a blob staged nothing: skip it)
+        const bool run = blob && H.ok && H.status == 0 && H.count > 0;
+        if (blob && !H.ok && tid == 0) set_status(blob, LQ_DEV_CORRUPT);
         TileReg<D> P;
         if (run) {
             const int8_t *c8 = reinterpret_cast<const int8_t *>(st + L.codes_off);
@@ -791,9 +802,9 @@ __global__ void __launch_bounds__(kGroup, 2) flush_kernel(FlushArgs A) {
         }
         gsync();  // the stage has been read
         if (refill) {
-            const uint32_t bytes = staged_bytes(L, F.window, c_next);
+            const uint32_t bytes = blob_next ? staged_bytes(L, F.window, c_next) : 0u;
             mbar_arrive_expect_tx(&full[s], bytes);
-            bulk_g2s(stages + (size_t)s * SB, blob_at(it + kFlushStages), bytes, &full[s]);
+            if (blob_next) bulk_g2s(stages + (size_t)s * SB, blob_next, bytes, &full[s]);
         }
         if (run) {
             const int ncomp = compress_tile<D, BITS>(P, F, L, scratch, blob, tid);
@@ -807,10 +818,12 @@ template <int D, int BITS, int MODE>
 __global__ void __launch_bounds__(kGroup) boundary_kernel(FlushArgs A) {
     constexpr int IP = FT<D>::IP, TJ = FT<D>::TJ;
     const int tid = threadIdx.x;
-    const size_t head = blockIdx.x;
+    const size_t head = blockIdx.x;  // work item: inputs and outputs are indexed by it
     const Layout L = A.L;
     const Flags F = A.F;
-    uint8_t *blob = A.state + head * L.blob;
+    const int bi = A.map.blob((int)head);
+    if (bi < 0) return;  // slot out of range: nothing to do (uniform over the CTA)
+    uint8_t *blob = A.state + (size_t)bi * L.blob;
     const Tile<D> tl(tid);
     const int i0 = tl.i0, j0 = tl.j0;
 

@@ -100,3 +100,37 @@ def test_status_strings(B):
     for code in range(9):
         assert B.lq_status_string(code)
     assert B.lq_status_string(99) == "unknown status"
+
+
+def test_slot_entry_points_rejected_before_launch(B):
+    cfg = B.make_config(4, 4)
+    L = B.lib
+    c = ctypes.byref(cfg)
+    # an empty slot list launches nothing
+    assert L.lq_decode_step_slots(c, 256, None, 0, None, None, None, None, None, None, None) == 0
+    assert L.lq_window_flush_slots(c, 256, None, 0, None) == 0
+    assert L.lq_state_init_slots(c, 256, None, 0, None, None) == 0
+    assert L.lq_copy_slots(c, 256, 2, None, 512, 3, None, 0, None) == 0
+    # missing pointers, negative counts
+    assert L.lq_decode_step_slots(c, 256, None, 2, 16, 16, 16, 16, 16, 16, None) == 1
+    assert L.lq_decode_step_slots(c, 256, 64, 2, 16, 16, 16, 16, 16, None, None) == 1
+    assert L.lq_decode_step_slots(c, 256, 64, -1, 16, 16, 16, 16, 16, 16, None) == 1
+    assert L.lq_window_flush_slots(c, None, 64, 2, None) == 1
+    assert L.lq_state_init_slots(c, 256, 64, 2, None, None) == 1
+    assert L.lq_copy_slots(c, 256, 0, 64, 512, 3, 64, 1, None) == 1
+    assert L.lq_copy_slots(c, 256, 2, None, 512, 3, 64, 1, None) == 1
+    # alignment: slot list 4 B, state 256 B, S0 16 B
+    assert L.lq_decode_step_slots(c, 256, 66, 2, 16, 16, 16, 16, 16, 16, None) == 6
+    assert L.lq_window_flush_slots(c, 128, 64, 2, None) == 6
+    assert L.lq_state_init_slots(c, 256, 64, 2, 8, None) == 6
+    assert L.lq_copy_slots(c, 256, 2, 64, 384, 3, 64, 1, None) == 6
+    # only the LeapQuant formats run through a slot list
+    for other in (B.make_config(4, 4, bits=32), B.make_config(4, 4, bits=8, per_step=True)):
+        o = ctypes.byref(other)
+        assert L.lq_decode_step_slots(o, 256, 64, 2, 16, 16, 16, 16, 16, 16, None) == 2
+        assert L.lq_window_flush_slots(o, 256, 64, 2, None) == 2
+        assert L.lq_state_init_slots(o, 256, 64, 2, 16, None) == 2
+    # a bad config is reported first
+    bad = B.make_config(4, 4)
+    bad.window = 0
+    assert L.lq_copy_slots(ctypes.byref(bad), 256, 2, 64, 512, 3, 64, 1, None) == 1
