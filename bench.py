@@ -53,6 +53,8 @@ def parse_args():
     ap.add_argument("--no-baselines", action="store_true",
                     help="skip the naive per-step BF16 / FP8 / INT8 states")
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--mt-tokens", type=int, default=4,
+                    help="tokens per launch of the multi-token decode line (0: skip it)")
     ap.add_argument("--no-slots", action="store_true",
                     help="skip the serving path (decode and flush through a slot list)")
     ap.add_argument("--cpu-seconds", type=float, default=10.0)
@@ -82,6 +84,18 @@ def decode_bytes(wl, count):
     read = (f["hdr"] + f["meta"] + f["qs"] + f["sm"] + f["cvec"] + f["codes"] + count * f["pair"]
             + f["g"] + f["inputs"])
     write = f["out"] + f["pair"] + f["g"] + 8
+    return read + write
+
+
+def multi_decode_bytes(wl, count, T):
+    """Algorithmic bytes of one T-token decode launch for one head with
+    `count` pairs buffered before it: the compact state, the pairs and the
+    decay product are read once; every token reads its inputs and writes its
+    output and its pair."""
+    f = field_bytes(wl)
+    read = (f["hdr"] + f["meta"] + f["qs"] + f["sm"] + f["cvec"] + f["codes"] + count * f["pair"]
+            + f["g"] + T * f["inputs"])
+    write = T * (f["out"] + f["pair"]) + f["g"] + 8
     return read + write
 
 
@@ -324,6 +338,32 @@ class SlotArm(Arm):
             self.states[l].flush_slots(self.slots)
 
 
+class MultiArm(Arm):
+    """The same layers decoded T tokens per launch (lq_decode_steps): a
+    window is W / T launches per layer, inputs regrouped [batch, T, H, .]."""
+
+    NAMES = ("q", "k", "v", "beta", "decay")
+
+    def __init__(self, wl, layers_data, torch, B, tokens):
+        super().__init__(wl, layers_data, wl.bits, torch, B)
+        self.T = tokens
+        W = wl.window
+        self.chunks = [[{n: torch.stack([x[n][t0 + i] for i in range(tokens)], dim=1).contiguous()
+                         for n in self.NAMES} for t0 in range(0, W, tokens)] for x in self.inp]
+        self.mout = [torch.empty((W // tokens, wl.batch, tokens, wl.heads, wl.dv), dtype=torch.float32,
+                                 device="cuda") for _ in layers_data]
+        torch.cuda.synchronize()
+
+    def decode_all(self):
+        for c in range(self.wl.window // self.T):
+            for l in range(self.L):
+                x = self.chunks[l][c]
+                self.states[l].steps(self.T, x["q"], x["k"], x["v"], x["beta"], x["decay"], self.mout[l][c])
+
+    def launches_per_step(self):
+        return (self.wl.window // self.T) * self.L + self.L
+
+
 def time_arm(arm, steps, warmup, torch, dist, world):
     """Time `steps` window-steps; returns total ms (max over ranks) and the
     per-step decode / flush split from events recorded between the graphs."""
@@ -550,6 +590,28 @@ def main_ours(args):
             del armb
             torch.cuda.empty_cache()
         line["per_step_baselines"] = base
+
+    # ---- multi-token decode: T tokens per launch, the compact state read once
+    if args.mt_tokens > 1 and W % args.mt_tokens == 0:
+        T = args.mt_tokens
+        armm = MultiArm(wl, layers, torch, B, T)
+        armm.capture()
+        km = args.fp32_steps or max(4, args.steps // 4)
+        tm, dm, fm = time_arm(armm, km, max(3, args.warmup // 2), torch, dist, world)
+        status = max(st.check() for st in armm.states)
+        if status != 0:
+            raise RuntimeError(f"device status after the multi-token run: {B.STATUS_NAMES[status]}")
+        n_launch = km * (W // T) * L
+        mb = nh * sum(multi_decode_bytes(wl, c, T) for c in range(0, W, T)) / (W // T)
+        dm_ms = dm / n_launch
+        line["multi_token"] = {
+            "tokens_per_launch": T, "value": whole_job_rate(km * W * L * nh, world, tm),
+            "unit": "head-tokens/s", "steps": km, "decode_avg_launch_us": dm_ms * 1e3,
+            "decode_us_per_token": dm_ms * 1e3 / T, "algorithmic_bytes_per_launch": mb,
+            "achieved_gbs": mb / (dm_ms / 1e3) / 1e9, "frac": mb / (dm_ms / 1e3) / 1e9 / hbm,
+            "flush_avg_launch_us": fm / (km * L) * 1e3}
+        del armm
+        torch.cuda.empty_cache()
 
     # ---- the serving path: the same work through a slot list
     if not args.no_slots:

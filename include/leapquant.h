@@ -188,6 +188,24 @@ LQ_API lq_status lq_dequant_state(const lq_config *cfg, const void *state, float
  * device pointer; the read uses one strided device-to-host copy. */
 LQ_API lq_status lq_check_status(const lq_config *cfg, const void *state, lq_stream_t stream);
 
+/* T consecutive tokens for every (slot, head) in one launch (speculative
+ * verification, multi-token prediction): the compact state is read once for
+ * all T tokens.  Token t's output and pair equal those of the t-th of T
+ * lq_decode_step calls on the same inputs, bit for bit.
+ *   tokens  T, 1 <= T <= W (LQ_ERR_INVALID_ARG otherwise) and T <= 8
+ *           (LQ_ERR_UNSUPPORTED above)
+ *   q, k    [N, T, H, dk]  in_dtype   v [N, T, H, dv]  in_dtype
+ *   beta    [N, T, H] f32;  decay [N, T, H] f32 (GDN) or [N, T, H, dk] (KDA)
+ *   out     [N, T, H, dv] f32
+ * A (slot, head) whose window lacks room for T more pairs is skipped as a
+ * whole (LQ_DEV_WINDOW_FULL, zero outputs).  If token t fails its range
+ * check, tokens t.. of that (slot, head) are skipped (zero outputs) and the
+ * state keeps the pairs of tokens < t.  bits 8/6/4 only (others:
+ * LQ_ERR_UNSUPPORTED).  T = 1 is lq_decode_step. */
+LQ_API lq_status lq_decode_steps(const lq_config *cfg, void *state, int tokens, const void *q,
+                                 const void *k, const void *v, const float *beta, const float *decay,
+                                 float *out, lq_stream_t stream);
+
 /* ---- Serving: a subset of the sequences through a slot list ----------
  * A continuous-batching server keeps N sequence slots in one state buffer
  * and decodes, at each step, only the sequences that are running.  The
@@ -216,6 +234,13 @@ LQ_API lq_status lq_decode_step_slots(const lq_config *cfg, void *state, const i
                                       int n_active, const void *q, const void *k, const void *v,
                                       const float *beta, const float *decay, float *out,
                                       lq_stream_t stream);
+
+/* lq_decode_steps for the slots in `slots` (row n of the [n_active, T, ...]
+ * tensors belongs to slot slots[n]). */
+LQ_API lq_status lq_decode_steps_slots(const lq_config *cfg, void *state, const int32_t *slots,
+                                       int n_active, int tokens, const void *q, const void *k,
+                                       const void *v, const float *beta, const float *decay,
+                                       float *out, lq_stream_t stream);
 
 /* lq_window_flush for the slots in `slots` (slots reach their window
  * boundary at different steps when sequences join at different times). */

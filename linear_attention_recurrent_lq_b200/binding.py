@@ -18,8 +18,11 @@ LQ_OK = 0
 STATUS_NAMES = {0: "LQ_OK", 1: "LQ_ERR_INVALID_ARG", 2: "LQ_ERR_UNSUPPORTED", 3: "LQ_ERR_CUDA",
                 4: "LQ_ERR_WINDOW_FULL", 5: "LQ_ERR_RANGE", 6: "LQ_ERR_MISALIGNED",
                 7: "LQ_ERR_TIMEOUT", 8: "LQ_ERR_CORRUPT"}
+(LQ_ERR_INVALID_ARG, LQ_ERR_UNSUPPORTED, LQ_ERR_CUDA, LQ_ERR_WINDOW_FULL, LQ_ERR_RANGE,
+ LQ_ERR_MISALIGNED, LQ_ERR_TIMEOUT, LQ_ERR_CORRUPT) = range(1, 9)
 ENTRY_POINTS = ("lq_validate_config", "lq_state_bytes", "lq_state_init", "lq_decode_step",
-                "lq_window_flush", "lq_dequant_state", "lq_check_status", "lq_state_init_slots",
+                "lq_window_flush", "lq_dequant_state", "lq_check_status", "lq_decode_steps",
+                "lq_state_init_slots", "lq_decode_steps_slots",
                 "lq_decode_step_slots", "lq_window_flush_slots", "lq_copy_slots", "lq_status_string")
 
 
@@ -85,6 +88,10 @@ def _load():
     L.lq_window_flush_slots.argtypes = [P, vp, vp, i32, vp]
     L.lq_window_flush_slots.restype = st
     L.lq_copy_slots.argtypes = [P, vp, i32, vp, vp, i32, vp, i32, vp]
+    L.lq_decode_steps.argtypes = [P, vp, i32, vp, vp, vp, vp, vp, vp, vp]
+    L.lq_decode_steps.restype = st
+    L.lq_decode_steps_slots.argtypes = [P, vp, vp, i32, i32, vp, vp, vp, vp, vp, vp, vp]
+    L.lq_decode_steps_slots.restype = st
     L.lq_copy_slots.restype = st
     L.lq_status_string.argtypes = [st]
     L.lq_status_string.restype = ctypes.c_char_p
@@ -175,6 +182,17 @@ def lq_decode_step_slots(cfg, state, slots, q, k, v, beta, decay, out, stream=No
                                     _stream(stream)), "lq_decode_step_slots")
 
 
+def lq_decode_steps(cfg, state, tokens, q, k, v, beta, decay, out, stream=None):
+    _check(lib.lq_decode_steps(ctypes.byref(cfg), _ptr(state), int(tokens), _ptr(q), _ptr(k), _ptr(v),
+                               _ptr(beta), _ptr(decay), _ptr(out), _stream(stream)), "lq_decode_steps")
+
+
+def lq_decode_steps_slots(cfg, state, slots, tokens, q, k, v, beta, decay, out, stream=None):
+    _check(lib.lq_decode_steps_slots(ctypes.byref(cfg), _ptr(state), _ptr(slots), _n(slots), int(tokens),
+                                     _ptr(q), _ptr(k), _ptr(v), _ptr(beta), _ptr(decay), _ptr(out),
+                                     _stream(stream)), "lq_decode_steps_slots")
+
+
 def lq_window_flush_slots(cfg, state, slots, stream=None):
     _check(lib.lq_window_flush_slots(ctypes.byref(cfg), _ptr(state), _ptr(slots), _n(slots),
                                      _stream(stream)), "lq_window_flush_slots")
@@ -215,6 +233,10 @@ class LQState:
     def flush(self, stream=None):
         lq_window_flush(self.cfg, self.buf, stream)
 
+    def steps(self, tokens, q, k, v, beta, decay, out, stream=None):
+        """T tokens per (slot, head): inputs [N, T, H, .], out [N, T, H, dv]."""
+        lq_decode_steps(self.cfg, self.buf, tokens, q, k, v, beta, decay, out, stream)
+
     def dequant(self, S_out=None, stream=None):
         import torch
         c = self.cfg
@@ -233,6 +255,9 @@ class LQState:
 
     def step_slots(self, slots, q, k, v, beta, decay, out, stream=None):
         lq_decode_step_slots(self.cfg, self.buf, slots, q, k, v, beta, decay, out, stream)
+
+    def steps_slots(self, slots, tokens, q, k, v, beta, decay, out, stream=None):
+        lq_decode_steps_slots(self.cfg, self.buf, slots, tokens, q, k, v, beta, decay, out, stream)
 
     def flush_slots(self, slots, stream=None):
         lq_window_flush_slots(self.cfg, self.buf, slots, stream)

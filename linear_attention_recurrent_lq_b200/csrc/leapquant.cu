@@ -118,8 +118,10 @@ int persistent_grid(K kernel, int threads, uint32_t smem, int work) {
 
 template <int D, int BITS>
 lq_status launch_decode(const lq_config &c, const DecodeArgs &a, cudaStream_t s) {
-    const uint32_t smem = decode_smem_bytes(D, a.L, a.F);
-    auto k = a.map.slots ? decode_kernel<D, BITS, true> : decode_kernel<D, BITS, false>;
+    const bool multi = a.tokens > 1;
+    const uint32_t smem = decode_smem_bytes(D, a.L, a.F, multi ? a.tokens : 1);
+    auto k = a.map.slots ? (multi ? decode_kernel<D, BITS, true, true> : decode_kernel<D, BITS, true, false>)
+                         : (multi ? decode_kernel<D, BITS, false, true> : decode_kernel<D, BITS, false, false>);
     cudaError_t e = allow_smem(k, smem);
     if (e != cudaSuccess) return LQ_ERR_CUDA;
     const int threads = D + 64;
@@ -292,7 +294,7 @@ lq_status lq_decode_step(const lq_config *cfg, void *state, const void *q, const
         return c.dk == 128 ? launch_fp32_decode<128>(c, a, s) : launch_fp32_decode<64>(c, a, s);
     }
     DecodeArgs a{static_cast<uint8_t *>(state), L, make_flags(c), q, k, v, beta, decay, out,
-                 c.num_slots * c.num_heads};
+                 c.num_slots * c.num_heads, SlotMap{nullptr, c.num_heads, c.num_slots}, 1};
     return dispatch_decode(c, a, s);
 }
 
@@ -386,8 +388,45 @@ lq_status lq_decode_step_slots(const lq_config *cfg, void *state, const int32_t 
     if (n_active == 0) return LQ_OK;
     const lq_config &c = *cfg;
     DecodeArgs a{static_cast<uint8_t *>(state), make_layout(c), make_flags(c), q, k, v, beta, decay, out,
-                 n_active * c.num_heads, SlotMap{slots, c.num_heads, c.num_slots}};
+                 n_active * c.num_heads, SlotMap{slots, c.num_heads, c.num_slots}, 1};
     return dispatch_decode(c, a, reinterpret_cast<cudaStream_t>(stream));
+}
+
+// T tokens per (slot, head) in one launch: the plain or slot-list kernel for
+// T = 1, the multi-token instance above.
+static lq_status decode_tokens(const lq_config *cfg, void *state, const int32_t *slots, int rows, int tokens,
+                               const void *q, const void *k, const void *v, const float *beta,
+                               const float *decay, float *out, lq_stream_t stream) {
+    const lq_config &c = *cfg;
+    if (tokens < 1 || tokens > c.window) return LQ_ERR_INVALID_ARG;
+    if (tokens > kMaxTokens) return LQ_ERR_UNSUPPORTED;
+    if (c.bits == 32 || c.per_step) return LQ_ERR_UNSUPPORTED;
+    if ((int64_t)rows * tokens * c.num_heads > 0x7FFFFFFF) return LQ_ERR_UNSUPPORTED;
+    if (rows > 0 && (!q || !k || !v || !beta || !decay || !out)) return LQ_ERR_INVALID_ARG;
+    if (!aligned(q, 16) || !aligned(k, 16) || !aligned(v, 16) || !aligned(beta, 4) ||
+        !aligned(decay, c.decay_kind ? 16 : 4) || !aligned(out, 4))
+        return LQ_ERR_MISALIGNED;
+    if (rows == 0) return LQ_OK;
+    DecodeArgs a{static_cast<uint8_t *>(state), make_layout(c), make_flags(c), q, k, v, beta, decay, out,
+                 rows * c.num_heads, SlotMap{slots, c.num_heads, c.num_slots}, tokens};
+    return dispatch_decode(c, a, reinterpret_cast<cudaStream_t>(stream));
+}
+
+lq_status lq_decode_steps(const lq_config *cfg, void *state, int tokens, const void *q, const void *k,
+                          const void *v, const float *beta, const float *decay, float *out, lq_stream_t stream) {
+    lq_status st = check_config(cfg);
+    if (st != LQ_OK) return st;
+    if (!state) return LQ_ERR_INVALID_ARG;
+    if (!aligned(state, 256)) return LQ_ERR_MISALIGNED;
+    return decode_tokens(cfg, state, nullptr, cfg->num_slots, tokens, q, k, v, beta, decay, out, stream);
+}
+
+lq_status lq_decode_steps_slots(const lq_config *cfg, void *state, const int32_t *slots, int n_active, int tokens,
+                                const void *q, const void *k, const void *v, const float *beta,
+                                const float *decay, float *out, lq_stream_t stream) {
+    lq_status st = check_slots(cfg, state, slots, n_active);
+    if (st != LQ_OK) return st;
+    return decode_tokens(cfg, state, slots, n_active, tokens, q, k, v, beta, decay, out, stream);
 }
 
 lq_status lq_window_flush_slots(const lq_config *cfg, void *state, const int32_t *slots, int n_active,

@@ -47,25 +47,30 @@ struct DecodeArgs {
     const float *beta, *decay;
     float *out;
     int num_heads;  // work items: N * H, or active rows * H with a slot map
-    SlotMap map;
+    SlotMap map;    // heads = H always; slots only in the slot-list instance
+    int tokens;     // T consecutive tokens per work item (multi-token instance)
 };
 
 constexpr int kDotSlots = kMaxWindow + kMaxComp;
+constexpr int kMaxTokens = 8;  // tokens per work item in one multi-token launch
 
-// One ring stage: [blob prefix up to the codes][buffered pairs][q k v][KDA decay][aux]
+// One ring stage: [blob prefix up to the codes][buffered pairs][q k v per
+// token][KDA decay per token][aux].  aux: f32 [0] 1 = the work item has no
+// blob, [4 + t] beta of token t, [4 + T + t] GDN alpha of token t.
 struct DecodeStage {
     uint32_t pairs_at, in_off, qkv_bytes, dec_off, aux_off, bytes;
 };
 
 __host__ __device__ inline DecodeStage decode_stage(const Layout &L, int D, int window, int bf16,
-                                                    int kda) {
+                                                    int kda, int tokens = 1) {
     DecodeStage S;
     S.pairs_at = L.codes_off;  // the prefix [0, codes_off) is copied as is
+    // pairs buffered before the launch plus those its earlier tokens append: at most W - 1
     S.in_off = align_up(S.pairs_at + (uint32_t)(window - 1) * L.pair_bytes, 128);
     S.qkv_bytes = align_up((uint32_t)D * (bf16 ? 2u : 4u), 16);
-    S.dec_off = S.in_off + 3 * S.qkv_bytes;
-    S.aux_off = align_up(S.dec_off + (kda ? (uint32_t)D * 4u : 0u), 16);
-    S.bytes = align_up(S.aux_off + 16, 128);
+    S.dec_off = S.in_off + 3u * S.qkv_bytes * (uint32_t)tokens;
+    S.aux_off = align_up(S.dec_off + (kda ? (uint32_t)D * 4u * (uint32_t)tokens : 0u), 16);
+    S.bytes = align_up(S.aux_off + 16 + 8 * (uint32_t)tokens, 128);
     return S;
 }
 
@@ -84,7 +89,7 @@ constexpr int kInfoRun = 0, kInfoCount = 1, kInfoNrow = 2, kInfoNcol = 3, kInfoB
 
 template <int D>
 __host__ __device__ constexpr uint32_t decode_fixed_smem() {
-    // barriers + control (128) | chunk sums float2 [D/16][D+1] | prep buffers [2]
+    // barriers (6 x 8 at 0, 2 more at 64) + control (128) | chunk sums float2 [D/16][D+1] | prep buffers [2]
     // | dots float2 [kDotSlots] | producer batch [4*32]
     return align_up(128u + 8u * (D / 16) * (D + 1) + 2u * PrepBuf<D>::bytes + 8u * kDotSlots + 4u * 32u * 4u,
                     128u);
@@ -94,9 +99,9 @@ constexpr int kDecodeStages = 2;
 // Prep-warp marker of a work item whose slot is out of range (never a status bit).
 constexpr uint32_t kSkipItem = 0xFFFFFFFFu;
 
-inline uint32_t decode_smem_bytes(int D, const Layout &L, const Flags &F) {
+inline uint32_t decode_smem_bytes(int D, const Layout &L, const Flags &F, int tokens = 1) {
     const uint32_t fixed = D == 128 ? decode_fixed_smem<128>() : decode_fixed_smem<64>();
-    return fixed + (uint32_t)kDecodeStages * decode_stage(L, D, F.window, F.bf16_in, F.kda).bytes;
+    return fixed + (uint32_t)kDecodeStages * decode_stage(L, D, F.window, F.bf16_in, F.kda, tokens).bytes;
 }
 
 __device__ __forceinline__ void consumer_sync(int n) {
@@ -240,10 +245,13 @@ __device__ __forceinline__ float warp_sum(float x) {
     return x;
 }
 
-// SLOTS: work items reach their blobs through A.map (a separate instance, so
-// the plain path carries none of the lookups).
-template <int D, int BITS, bool SLOTS>
-__global__ void __launch_bounds__(D + 64, SLOTS ? 3 : 0) decode_kernel(DecodeArgs A) {
+// SLOTS: work items reach their blobs through A.map.  MULTI: each work item
+// takes A.tokens consecutive tokens (inputs and outputs [rows, T, H, .]),
+// reading its compact state once; token t sees the pairs of tokens < t
+// through the stage, where the epilogue also appends them.  Separate
+// instances, so the plain path carries none of this.
+template <int D, int BITS, bool SLOTS, bool MULTI>
+__global__ void __launch_bounds__(D + 64, (SLOTS || MULTI) ? 3 : 0) decode_kernel(DecodeArgs A) {
     constexpr int NC = D;            // consumer threads
     constexpr int LPR = D / 16;      // threads per row, one 16-key chunk each
     constexpr int RPT = D / 16;      // rows per thread (16 row groups)
@@ -260,15 +268,23 @@ __global__ void __launch_bounds__(D + 64, SLOTS ? 3 : 0) decode_kernel(DecodeArg
     const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
     const Layout L = A.L;
     const Flags F = A.F;
-    const DecodeStage SG = decode_stage(L, D, F.window, F.bf16_in, F.kda);
+    const int T = MULTI ? A.tokens : 1;
+    const DecodeStage SG = decode_stage(L, D, F.window, F.bf16_in, F.kda, T);
     const int G = gridDim.x;
     const int n_mine = (A.num_heads - (int)blockIdx.x + G - 1) / G;
     auto blob_of = [](const SlotMap &m, int h) { return SLOTS ? m.blob(h) : h; };
+    // input / output row of token t of work item h: ((h / H) T + t) H + h % H
+    auto tok_row = [&](size_t h, int t) -> size_t {
+        if (!MULTI) return h;
+        const int H = A.map.heads;
+        return h + ((size_t)((int)h / H) * (size_t)(T - 1) + (size_t)t) * (size_t)H;
+    };
 
     extern __shared__ __align__(128) uint8_t smem[];
     uint64_t *full = reinterpret_cast<uint64_t *>(smem);  // [2] stage landed
     uint64_t *empty = full + 2;                           // [2] consumers done with the stage
-    uint64_t *pfull = empty + 2;                          // [2] prep of the head done
+    uint64_t *pfull = empty + 2;                          // [2] prep of the step done
+    uint64_t *pempty = reinterpret_cast<uint64_t *>(smem + 64);  // [2] consumers done with a prep buffer (MULTI)
     volatile uint32_t *s_abort = reinterpret_cast<volatile uint32_t *>(smem + 120);
     float2 *s_part = reinterpret_cast<float2 *>(smem + 128);            // chunk sums [LPR][PSTR]
     uint8_t *s_pb = reinterpret_cast<uint8_t *>(s_part + LPR * PSTR);    // PrepBuf [2]
@@ -284,6 +300,7 @@ __global__ void __launch_bounds__(D + 64, SLOTS ? 3 : 0) decode_kernel(DecodeArg
             mbar_init(&full[s], 1);
             mbar_init(&empty[s], NC / 32);  // one arrival per consumer warp
             mbar_init(&pfull[s], 32);       // every lane of the prep warp
+            if (MULTI) mbar_init(&pempty[s], NC / 32);
         }
         *s_abort = 0u;
         fence_mbar_init();
@@ -311,8 +328,10 @@ __global__ void __launch_bounds__(D + 64, SLOTS ? 3 : 0) decode_kernel(DecodeArg
                 const int b = blob_of(A.map, (int)h);
                 s_bidx[lane] = (int)b;
                 s_cnt[lane] = b >= 0 ? *reinterpret_cast<const uint32_t *>(A.state + b * L.blob + kHdrCount) : 0u;
-                s_pbeta[lane] = A.beta[h];
-                s_palpha[lane] = F.kda ? 1.f : A.decay[h];
+                if (!MULTI) {
+                    s_pbeta[lane] = A.beta[h];
+                    s_palpha[lane] = F.kda ? 1.f : A.decay[h];
+                }
             }
             __syncwarp();
             if (lane == 0) {
@@ -326,9 +345,26 @@ __global__ void __launch_bounds__(D + 64, SLOTS ? 3 : 0) decode_kernel(DecodeArg
                     const size_t h = blockIdx.x + (size_t)it * G;
                     uint8_t *st = stages + (size_t)s * SG.bytes;
                     float *aux = reinterpret_cast<float *>(st + SG.aux_off);
-                    aux[0] = s_pbeta[x];
-                    aux[1] = s_palpha[x];
-                    aux[2] = s_bidx[x] >= 0 ? 0.f : 1.f;  // 1: no blob for this work item
+                    if (!MULTI) {
+                        aux[4] = s_pbeta[x];
+                        aux[5] = s_palpha[x];
+                    } else {
+                        float bt[kMaxTokens], at[kMaxTokens];
+#pragma unroll
+                        for (int t = 0; t < kMaxTokens; ++t)
+                            if (t < T) {
+                                const size_t r = tok_row(h, t);
+                                bt[t] = A.beta[r];
+                                at[t] = F.kda ? 1.f : A.decay[r];
+                            }
+#pragma unroll
+                        for (int t = 0; t < kMaxTokens; ++t)
+                            if (t < T) {
+                                aux[4 + t] = bt[t];
+                                aux[4 + T + t] = at[t];
+                            }
+                    }
+                    aux[0] = s_bidx[x] >= 0 ? 0.f : 1.f;  // 1: no blob for this work item
                     if (s_bidx[x] < 0) {
                         mbar_arrive_expect_tx(&full[s], 0u);  // nothing is staged
                         continue;
@@ -337,17 +373,21 @@ __global__ void __launch_bounds__(D + 64, SLOTS ? 3 : 0) decode_kernel(DecodeArg
                     const uint32_t c = s_cnt[x];
                     const uint32_t cc = c < (uint32_t)F.window ? c : 0u;
                     const uint32_t pb = cc * L.pair_bytes;
-                    mbar_arrive_expect_tx(&full[s], L.codes_off + pb + 3 * SG.qkv_bytes +
-                                                        (F.kda ? (uint32_t)D * 4u : 0u));
+                    mbar_arrive_expect_tx(&full[s], L.codes_off + pb +
+                                                        (uint32_t)T * (3 * SG.qkv_bytes + (F.kda ? (uint32_t)D * 4u : 0u)));
                     bulk_g2s(st, blob, L.codes_off, &full[s]);
                     if (pb) bulk_g2s(st + SG.pairs_at, blob + L.pairs_off, pb, &full[s]);
-                    const size_t qo = h * (size_t)SG.qkv_bytes;
-                    bulk_g2s(st + SG.in_off, static_cast<const uint8_t *>(A.q) + qo, SG.qkv_bytes, &full[s]);
-                    bulk_g2s(st + SG.in_off + SG.qkv_bytes, static_cast<const uint8_t *>(A.k) + qo,
-                             SG.qkv_bytes, &full[s]);
-                    bulk_g2s(st + SG.in_off + 2 * SG.qkv_bytes, static_cast<const uint8_t *>(A.v) + qo,
-                             SG.qkv_bytes, &full[s]);
-                    if (F.kda) bulk_g2s(st + SG.dec_off, A.decay + h * D, (uint32_t)D * 4u, &full[s]);
+                    for (int t = 0; t < T; ++t) {
+                        const size_t r = tok_row(h, t);
+                        const size_t qo = r * (size_t)SG.qkv_bytes;
+                        uint8_t *in = st + SG.in_off + (size_t)t * 3 * SG.qkv_bytes;
+                        bulk_g2s(in, static_cast<const uint8_t *>(A.q) + qo, SG.qkv_bytes, &full[s]);
+                        bulk_g2s(in + SG.qkv_bytes, static_cast<const uint8_t *>(A.k) + qo, SG.qkv_bytes, &full[s]);
+                        bulk_g2s(in + 2 * SG.qkv_bytes, static_cast<const uint8_t *>(A.v) + qo, SG.qkv_bytes,
+                                 &full[s]);
+                        if (F.kda)
+                            bulk_g2s(st + SG.dec_off + (size_t)t * D * 4, A.decay + r * D, (uint32_t)D * 4u, &full[s]);
+                    }
                 }
             }
             __syncwarp();
@@ -361,14 +401,23 @@ __global__ void __launch_bounds__(D + 64, SLOTS ? 3 : 0) decode_kernel(DecodeArg
         // lists, the new decay product, y = g . k and g . q, the new key in
         // the window-start frame, x = sm . y quantized per 16-key chunk to
         // int16, and k . q.  Lane l takes keys KPL*l .. KPL*l + KPL - 1.
-        for (int it = 0; it < n_mine; ++it) {
+        // One step per (head, token); the decay product runs on in registers
+        // over the tokens of a head.
+        float gprev[KPL];
+        bool dead = false;  // a token of this head failed its range check
+        for (int step = 0; step < n_mine * T; ++step) {
+            const int it = MULTI ? step / T : step, t = MULTI ? step - it * T : 0;
             const int s = it % kDecodeStages;
             const uint8_t *st = stages + (size_t)s * SG.bytes;
-            uint8_t *pb = s_pb + (it & 1) * PB::bytes;
+            uint8_t *pb = s_pb + (step & 1) * PB::bytes;
             uint32_t *info = reinterpret_cast<uint32_t *>(pb + PB::info);
-            if (!mbar_wait_bounded(&full[s], (uint32_t)(it / kDecodeStages) & 1u)) {
+            if (t == 0 && !mbar_wait_bounded(&full[s], (uint32_t)(it / kDecodeStages) & 1u)) {
                 if (lane == 0) *s_abort = 1u;
                 break;  // the consumers time out on their own wait
+            }
+            if (MULTI && step >= 2 && !mbar_wait_bounded(&pempty[step & 1], (uint32_t)((step >> 1) - 1) & 1u)) {
+                if (lane == 0) *s_abort = 1u;
+                break;
             }
             const uint4 hdr = *reinterpret_cast<const uint4 *>(st);  // count, status, ncomp, magic
             const uint32_t ncomp = hdr.z;
@@ -384,32 +433,40 @@ __global__ void __launch_bounds__(D + 64, SLOTS ? 3 : 0) decode_kernel(DecodeArg
             uint32_t newbits = 0;
             if (hdr.w != kMagic || ncomp > (uint32_t)F.num_comp || hdr.x > (uint32_t)F.window || badm)
                 newbits = LQ_DEV_CORRUPT;
-            else if (hdr.y == 0 && hdr.x >= (uint32_t)F.window)
-                newbits = LQ_DEV_WINDOW_FULL;
+            else if (hdr.y == 0 && hdr.x + (uint32_t)T > (uint32_t)F.window)
+                newbits = LQ_DEV_WINDOW_FULL;  // the window has no room for the T pairs
             // a work item without a blob: the stage holds stale bytes, skip it
-            if (reinterpret_cast<const float *>(st + SG.aux_off)[2] != 0.f) newbits = kSkipItem;
-            bool run = hdr.y == 0 && newbits == 0;
+            if (reinterpret_cast<const float *>(st + SG.aux_off)[0] != 0.f) newbits = kSkipItem;
+            if (t == 0) dead = false;
+            bool run = hdr.y == 0 && newbits == 0 && !dead;
             if (newbits == kSkipItem) newbits = 0;
             float kq = 0.f;
             if (run) {
                 const int i0 = KPL * lane;
+                const uint8_t *in = st + SG.in_off + (size_t)t * 3 * SG.qkv_bytes;
                 float kv[KPL], qv[KPL], gn[KPL];
 #pragma unroll
                 for (int e = 0; e < KPL; ++e) {
-                    kv[e] = load_in(st + SG.in_off + SG.qkv_bytes, i0 + e, F.bf16_in);
-                    qv[e] = load_in(st + SG.in_off, i0 + e, F.bf16_in);
+                    kv[e] = load_in(in + SG.qkv_bytes, i0 + e, F.bf16_in);
+                    qv[e] = load_in(in, i0 + e, F.bf16_in);
                 }
-                if (F.kda) {
+                if (t == 0) {
 #pragma unroll
                     for (int e = 0; e < KPL; ++e)
-                        gn[e] = reinterpret_cast<const float *>(st + L.g_off)[i0 + e] *
-                                reinterpret_cast<const float *>(st + SG.dec_off)[i0 + e];
-                } else {
-                    const float gs = *reinterpret_cast<const float *>(st + kHdrG) *
-                                     reinterpret_cast<const float *>(st + SG.aux_off)[1];
-#pragma unroll
-                    for (int e = 0; e < KPL; ++e) gn[e] = gs;
+                        gprev[e] = F.kda ? reinterpret_cast<const float *>(st + L.g_off)[i0 + e]
+                                         : *reinterpret_cast<const float *>(st + kHdrG);
                 }
+                if (F.kda) {
+                    const float *dec = reinterpret_cast<const float *>(st + SG.dec_off + (size_t)t * D * 4);
+#pragma unroll
+                    for (int e = 0; e < KPL; ++e) gn[e] = gprev[e] * dec[i0 + e];
+                } else {
+                    const float alpha = reinterpret_cast<const float *>(st + SG.aux_off)[4 + T + t];
+#pragma unroll
+                    for (int e = 0; e < KPL; ++e) gn[e] = gprev[e] * alpha;
+                }
+#pragma unroll
+                for (int e = 0; e < KPL; ++e) gprev[e] = gn[e];
                 bool bad = false;
                 float yk[KPL], yq[KPL], kh[KPL], xk[KPL], xq[KPL];
                 float mk = 0.f, mq = 0.f;
@@ -477,19 +534,20 @@ __global__ void __launch_bounds__(D + 64, SLOTS ? 3 : 0) decode_kernel(DecodeArg
                 kq = warp_sum(kq);
                 if (bad) {
                     run = false;
+                    dead = true;  // the later tokens of this head are skipped too
                     newbits = LQ_DEV_RANGE;
                 }
             }
             if (lane == 0) {
                 info[kInfoRun] = run ? 1u : 0u;
-                info[kInfoCount] = hdr.x;
+                info[kInfoCount] = hdr.x + (uint32_t)t;
                 info[kInfoNrow] = (uint32_t)__popc(rowm);
                 info[kInfoNcol] = (uint32_t)__popc(colm);
                 info[kInfoBits] = newbits;
                 info[kInfoKq] = __float_as_uint(kq);
             }
             __syncwarp();
-            mbar_arrive(&pfull[s]);
+            mbar_arrive(&pfull[step & 1]);
         }
         return;
     }
@@ -514,29 +572,32 @@ __global__ void __launch_bounds__(D + 64, SLOTS ? 3 : 0) decode_kernel(DecodeArg
     // the prep of the head), so the chunk sums and dot products of the
     // previous head are free by then; the stage goes back to the copy warp
     // when every consumer warp has arrived on its "empty" barrier.
-    for (int it = 0; it < n_mine; ++it) {
+    for (int step = 0; step < n_mine * T; ++step) {
+        const int it = MULTI ? step / T : step, t = MULTI ? step - it * T : 0;
         const int s = it % kDecodeStages;
-        const uint32_t ph = (uint32_t)(it / kDecodeStages) & 1u;
+        const uint32_t ph = (uint32_t)(step >> 1) & 1u;  // phase of this step's prep barrier
         const uint8_t *st = stages + (size_t)s * SG.bytes;
-        const uint8_t *pb = s_pb + (it & 1) * PB::bytes;
+        const uint8_t *pb = s_pb + (step & 1) * PB::bytes;
         const size_t h = blockIdx.x + (size_t)it * G;
+        const size_t orow = tok_row(h, t);  // input / output row of this token
         const int bi = blob_of(A.map, (int)h);
         uint8_t *blob = A.state + (bi >= 0 ? (size_t)bi : 0) * L.blob;
-        // codes of the next work item to load (through a slot map: if it has a blob)
-        bool has_next = it + 1 < n_mine;
+        // codes of the next work item to load, during the last token of this
+        // one (through a slot map: if it has a blob)
+        bool has_next = it + 1 < n_mine && t == T - 1;
         const uint8_t *next_codes = code_base + (h + G) * (size_t)L.blob;
         if constexpr (SLOTS) {
             const int bn = has_next ? A.map.blob((int)h + G) : -1;
             has_next = bn >= 0;
             next_codes = code_base + (size_t)(has_next ? bn : 0) * L.blob;
         }
-        if (!consumer_sync_and(mbar_wait_bounded(&pfull[s], ph), NC)) {
+        if (!consumer_sync_and(mbar_wait_bounded(&pfull[step & 1], ph), NC)) {
             // the data never arrived: record it on this blob and stop this CTA
             if (tid == 0) {
                 if (bi >= 0) set_status(blob, LQ_DEV_TIMEOUT);
                 *s_abort = 1u;
             }
-            A.out[h * D + tid] = 0.f;
+            A.out[orow * D + tid] = 0.f;
             break;
         }
         const uint32_t *info = reinterpret_cast<const uint32_t *>(pb + PB::info);
@@ -638,14 +699,21 @@ __global__ void __launch_bounds__(D + 64, SLOTS ? 3 : 0) decode_kernel(DecodeArg
                 const float uj = up[(size_t)m * 2 * D];
                 ab = __ffma2_rn(s_dot[m], make_float2(uj, uj), ab);
             }
-            const float u = aux[0] * (load_in(st + SG.in_off + 2 * SG.qkv_bytes, j, F.bf16_in) - ab.x);
+            const float u = aux[4 + t] * (load_in(st + SG.in_off + ((size_t)t * 3 + 2) * SG.qkv_bytes, j, F.bf16_in) - ab.x);
             const float kq = __uint_as_float(info[kInfoKq]);
-            A.out[h * D + j] = fmaf(kq, u, ab.y);
+            A.out[orow * D + j] = fmaf(kq, u, ab.y);
             const float *pkh = reinterpret_cast<const float *>(pb + PB::kh);
             const float *pg = reinterpret_cast<const float *>(pb + PB::g);
             float *pair = reinterpret_cast<float *>(blob + L.pairs_off + (size_t)count * L.pair_bytes);
             pair[D + j] = u;
             pair[tid] = pkh[tid];
+            if (MULTI && t < T - 1) {
+                // the later tokens of this head read the pair from the stage
+                float *sp = reinterpret_cast<float *>(const_cast<uint8_t *>(st) + SG.pairs_at +
+                                                      (size_t)count * L.pair_bytes);
+                sp[D + j] = u;
+                sp[tid] = pkh[tid];
+            }
             if (F.kda) reinterpret_cast<float *>(blob + L.g_off)[tid] = pg[tid];
             if (tid == 0) {
                 *reinterpret_cast<uint32_t *>(blob + kHdrCount) = count + 1;
@@ -657,11 +725,14 @@ __global__ void __launch_bounds__(D + 64, SLOTS ? 3 : 0) decode_kernel(DecodeArg
 #pragma unroll
                 for (int m = 0; m < RPT; ++m) load_group<BITS>(cg[m], next_codes + (size_t)(RPT * rg + m) * L.row_bytes);
             }
-            A.out[h * D + tid] = 0.f;
+            A.out[orow * D + tid] = 0.f;
             if (tid == 0 && newbits) set_status(blob, newbits);
         }
         __syncwarp();
-        if (lane == 0) mbar_arrive(&empty[s]);  // this warp is done with stage s
+        if (lane == 0) {
+            if (MULTI) mbar_arrive(&pempty[step & 1]);  // this warp is done with the prep buffer
+            if (t == T - 1) mbar_arrive(&empty[s]);     // ... and, after the last token, with stage s
+        }
     }
 }
 

@@ -134,3 +134,23 @@ def test_slot_entry_points_rejected_before_launch(B):
     bad = B.make_config(4, 4)
     bad.window = 0
     assert L.lq_copy_slots(ctypes.byref(bad), 256, 2, 64, 512, 3, 64, 1, None) == 1
+
+
+def test_multi_token_arguments_rejected_before_launch(B):
+    cfg = B.make_config(4, 4, window=16)
+    L = B.lib
+    c = ctypes.byref(cfg)
+    ok = (16, 16, 16, 16, 16, 16)
+    assert L.lq_decode_steps(c, 256, 0, *ok, None) == 1          # T >= 1
+    assert L.lq_decode_steps(c, 256, 9, *ok, None) == 2          # T <= 8
+    small = B.make_config(4, 4, window=4)
+    assert L.lq_decode_steps(ctypes.byref(small), 256, 5, *ok, None) == 1  # T <= W
+    assert L.lq_decode_steps(c, None, 2, *ok, None) == 1
+    assert L.lq_decode_steps(c, 128, 2, *ok, None) == 6
+    assert L.lq_decode_steps(c, 256, 2, 16, 16, 16, 16, 16, None, None) == 1
+    assert L.lq_decode_steps(c, 256, 2, 8, 16, 16, 16, 16, 16, None) == 6
+    for other in (B.make_config(4, 4, bits=32), B.make_config(4, 4, bits=16, per_step=True)):
+        assert L.lq_decode_steps(ctypes.byref(other), 256, 2, *ok, None) == 2
+    assert L.lq_decode_steps_slots(c, 256, 64, 0, 2, None, None, None, None, None, None, None) == 0
+    assert L.lq_decode_steps_slots(c, 256, None, 2, 2, *ok, None) == 1
+    assert L.lq_decode_steps_slots(c, 256, 64, 2, 9, *ok, None) == 2
