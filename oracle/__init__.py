@@ -78,6 +78,8 @@ def bind(path: str):
     L.lqo_run.restype = ctypes.c_int
     L.lqo_run.argtypes = [P(_Params), ctypes.c_int, ctypes.c_int, vp, vp, vp, vp, vp, vp,
                           vp, vp, ctypes.c_int]
+    L.lqo_prefill.restype = ctypes.c_int
+    L.lqo_prefill.argtypes = [ctypes.c_int] * 5 + [vp] * 9 + [ctypes.c_int]
     L.lqo_window_buffered.argtypes = [ctypes.c_int, ctypes.c_int, ctypes.c_int, vp, vp, vp,
                                       vp, vp, vp, vp, vp]
     L.lqo_round_f16.restype = ctypes.c_double
@@ -196,6 +198,32 @@ def run(p: Params, S0, q, k, v, beta, decay, threads: int = 0):
     used = lib().lqo_run(ctypes.byref(p.c()), nh, T, s0p, qp, kp, vp, bp, dp, o.ctypes.data,
                          S_end.ctypes.data, int(threads))
     return o, S_end, used
+
+
+def prefill(p: Params, S0, q, k, v, beta, decay, lengths=None, threads: int = 0):
+    """Prompt handoff: the FP64 delta rule over each head's prompt from S0,
+    then the FP32 rounding of the final state compressed as at a window
+    boundary.  Layouts as run(); lengths [nh] (None: all T).  Returns
+    (o [T, nh, dv] with zeros past a head's length, S_end [nh, dk, dv] FP64,
+    [compress(p, fl32(S_end[h])) for each head])."""
+    S0, s0p = _c(S0, np.float32)
+    nh = S0.shape[0]
+    q, qp = _c(q, np.float32)
+    T = q.shape[0]
+    k, kp = _c(k, np.float32)
+    v, vp = _c(v, np.float32)
+    beta, bp = _c(beta, np.float32)
+    decay, dp = _c(decay, np.float32)
+    assert q.shape == (T, nh, p.dk) and v.shape == (T, nh, p.dv) and beta.shape == (T, nh)
+    assert decay.shape == ((T, nh, p.dk) if p.kda else (T, nh))
+    lp = None
+    if lengths is not None:
+        lengths, lp = _c(np.asarray(lengths).reshape(nh), np.int32)
+    o = np.zeros((T, nh, p.dv), np.float64)
+    S_end = np.zeros((nh, p.dk, p.dv), np.float64)
+    lib().lqo_prefill(p.dk, p.dv, int(p.kda), nh, T, lp, s0p, qp, kp, vp, bp, dp, o.ctypes.data,
+                      S_end.ctypes.data, int(threads))
+    return o, S_end, [compress(p, S_end[h].astype(np.float32)) for h in range(nh)]
 
 
 def window_buffered(S_base, q, k, v, beta, a):

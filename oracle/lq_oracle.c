@@ -452,6 +452,51 @@ int lqo_run(const lqo_params *p, int nh, int T, const float *S0, const float *q,
     return used;
 }
 
+/* Prompt handoff.  [NEWS] per-window paragraph: the state a prefill leaves
+ * enters the quantized cache, and decoding starts from it.  Per head, the
+ * FP64 delta rule (lqo_step) over its first len[h] prompt tokens from S0;
+ * outputs of tokens at or past len[h] are 0.  S_end is the FP64 final state;
+ * the caller compresses its FP32 rounding (lqo_compress), as at a window
+ * boundary.  Layouts as lqo_run; len [nh] (NULL: all T).
+ * Returns the number of threads used.                                       */
+int lqo_prefill(int dk, int dv, int kda, int nh, int T, const int *len, const float *S0,
+                const float *q, const float *k, const float *v, const float *beta,
+                const float *decay, double *o, double *S_end, int threads)
+{
+    int used = 1;
+#ifdef _OPENMP
+    if (threads > 0) omp_set_num_threads(threads);
+#pragma omp parallel
+    {
+#pragma omp single
+        used = omp_get_num_threads();
+    }
+#endif
+#pragma omp parallel for schedule(dynamic, 1)
+    for (int h = 0; h < nh; ++h) {
+        double *S = S_end + (size_t)h * dk * dv;
+        double *qd = (double *)malloc(sizeof(double) * dk), *kd = (double *)malloc(sizeof(double) * dk);
+        double *vd = (double *)malloc(sizeof(double) * dv), *ad = (double *)malloc(sizeof(double) * dk);
+        double *od = (double *)malloc(sizeof(double) * dv);
+        const int n = len ? (len[h] < 0 ? 0 : (len[h] > T ? T : len[h])) : T;
+        for (int x = 0; x < dk * dv; ++x) S[x] = (double)S0[(size_t)h * dk * dv + x];
+        for (int t = 0; t < T; ++t) {
+            size_t th = (size_t)t * nh + h;
+            if (t >= n) {
+                for (int j = 0; j < dv; ++j) o[th * dv + j] = 0.0;
+                continue;
+            }
+            for (int i = 0; i < dk; ++i) { qd[i] = q[th * dk + i]; kd[i] = k[th * dk + i]; }
+            for (int j = 0; j < dv; ++j) vd[j] = v[th * dv + j];
+            for (int i = 0; i < dk; ++i) ad[i] = kda ? decay[th * dk + i] : decay[th];
+            lqo_step(dk, dv, S, qd, kd, vd, (double)beta[th], ad, od, NULL);
+            for (int j = 0; j < dv; ++j) o[th * dv + j] = od[j];
+        }
+        free(qd); free(kd); free(vd); free(ad); free(od);
+    }
+    return used;
+}
+
 /* The buffered window form, FP64, with explicit decay products (no
  * division): within a window starting from S_base,
  *   S'_t = P_t S_base + sum_{m<t} (Q_{m,t} k_m) u_m^T,   P_t = prod_{s<=t} D_s,

@@ -55,6 +55,12 @@ MUTATIONS = {
                                                "const float sc = (float)((double)m / 240.0);"),
     "fp8 scale per key row": ("for (int i = 0; i < dk; ++i) m = fmaxf(m, fabsf(S32[i * dv + j]));",
                               "for (int i = 0; i < dk; ++i) m = fmaxf(m, fabsf(S32[j * dv + i]));"),
+    "prefill ignores the prompt length": (
+        "const int n = len ? (len[h] < 0 ? 0 : (len[h] > T ? T : len[h])) : T;",
+        "const int n = T;"),
+    "prefill reads the decay of the wrong token": (
+        "ad[i] = kda ? decay[th * dk + i] : decay[th];",
+        "ad[i] = kda ? decay[(th % nh) * dk + i] : decay[th % nh];"),
     "per-step state not stored after the token": (
         "                per_step_store(p, S, buf32, qs, val);\n            } else",
         "                ;\n            } else"),

@@ -522,3 +522,76 @@ def test_naive_per_step_baselines_lose_more_than_leapquant(oracle_lib):
     assert e_bf16 < e_fp8, (e_bf16, e_fp8)
     # the table's headline: 8-bit LeapQuant also beats the per-step BF16 state
     assert e_lq < e_bf16, (e_lq, e_bf16)
+
+
+# --------------------------------------------------------------------------
+# prompt handoff (prefill, then the state enters the quantized cache)
+
+def test_prefill_matches_brute_force_on_tiny_heads(oracle_lib):
+    """The dense recurrence over the prompt and the compression of its FP32
+    rounding, against the independent NumPy restatement, per head with its
+    own prompt length."""
+    rng = np.random.default_rng(91)
+    for kda, bits, smoothing in ((False, 8, True), (True, 4, True), (False, 6, False)):
+        dk = dv = 16
+        T, nh, r = 11, 3, 2
+        lengths = [11, 0, 6]
+        S0 = np.stack([_rand_state(rng, dk, dv, rows=(1,), cols=(7,), gain=20.0) for _ in range(nh)])
+        S0 = S0.astype(np.float32)
+        q = rng.normal(size=(T, nh, dk)).astype(np.float32) / 4
+        k = rng.normal(size=(T, nh, dk)).astype(np.float32) / 4
+        v = rng.normal(size=(T, nh, dv)).astype(np.float32)
+        beta = rng.uniform(0.1, 0.9, (T, nh)).astype(np.float32)
+        a = rng.uniform(0.6, 1.0, (T, nh, dk) if kda else (T, nh)).astype(np.float32)
+        p = oracle.Params(dk=dk, dv=dv, window=4, num_comp=r, bits=bits, kda=kda, smoothing=smoothing)
+        o, S, comp = oracle.prefill(p, S0, q, k, v, beta, a, lengths=lengths)
+        for h in range(nh):
+            n = lengths[h]
+            ah = a[:, h] if kda else np.repeat(a[:, h:h + 1], dk, 1)
+            ob, Sb = brute.run(S0[h], q[:n, h], k[:n, h], v[:n, h], beta[:n, h], ah[:n], 4, 32, r,
+                               smoothing)
+            if n:
+                np.testing.assert_allclose(o[:n, h], ob, rtol=1e-9, atol=1e-12)
+            assert not o[n:, h].any()
+            np.testing.assert_allclose(S[h], Sb, rtol=1e-9, atol=1e-12)
+            cb = brute.compress(Sb.astype(np.float32), bits, r, smoothing)
+            np.testing.assert_array_equal(comp[h]["codes"], cb["codes"])
+            np.testing.assert_array_equal(comp[h]["qs"], cb["qs"])
+            np.testing.assert_array_equal(comp[h]["sm"], cb["sm"])
+
+
+def test_prefill_without_writes_is_pure_decay(oracle_lib):
+    """beta = 0: nothing is written, so after t tokens the state is the decay
+    product times S0 (powers of two keep it exact) and o_t = S_t^T q_t."""
+    rng = np.random.default_rng(92)
+    dk, dv, T = 8, 6, 5
+    S0 = rng.normal(size=(1, dk, dv)).astype(np.float32)
+    q = rng.normal(size=(T, 1, dk)).astype(np.float32)
+    k = rng.normal(size=(T, 1, dk)).astype(np.float32)
+    v = rng.normal(size=(T, 1, dv)).astype(np.float32)
+    beta = np.zeros((T, 1), np.float32)
+    for kda in (False, True):
+        a = (2.0 ** -rng.integers(0, 3, (T, 1, dk)) if kda else 2.0 ** -rng.integers(0, 3, (T, 1)))
+        a = a.astype(np.float32)
+        p = oracle.Params(dk=dk, dv=dv, num_comp=1, kda=kda)
+        o, S, _ = oracle.prefill(p, S0, q, k, v, beta, a)
+        G = np.ones(dk)
+        for t in range(T):
+            G = G * a[t, 0]
+            St = G[:, None] * S0[0].astype(np.float64)
+            np.testing.assert_allclose(o[t, 0], St.T @ q[t, 0].astype(np.float64), rtol=1e-13, atol=1e-13)
+        np.testing.assert_array_equal(S[0], G[:, None] * S0[0].astype(np.float64))
+
+
+def test_prefill_one_token_from_zero_writes_beta_k_v(oracle_lib):
+    """From a zero state one token leaves S = beta k v^T (u = beta v, nothing
+    to subtract) and o = beta (k . q) v: the orientation of the update."""
+    dk, dv = 4, 3
+    k = np.array([[[1.0, 2.0, 0.0, -1.0]]], np.float32)
+    q = np.array([[[0.5, 0.0, 1.0, 2.0]]], np.float32)
+    v = np.array([[[3.0, -1.0, 2.0]]], np.float32)
+    p = oracle.Params(dk=dk, dv=dv, num_comp=0)
+    o, S, _ = oracle.prefill(p, np.zeros((1, dk, dv), np.float32), q, k, v,
+                             np.array([[0.5]], np.float32), np.array([[0.75]], np.float32))
+    np.testing.assert_array_equal(S[0], 0.5 * np.outer(k[0, 0], v[0, 0]))
+    np.testing.assert_array_equal(o[0, 0], 0.5 * float(k[0, 0] @ q[0, 0]) * v[0, 0])
