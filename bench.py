@@ -55,6 +55,8 @@ def parse_args():
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--mt-tokens", type=int, default=4,
                     help="tokens per launch of the multi-token decode line (0: skip it)")
+    ap.add_argument("--prefill-tokens", type=int, default=256,
+                    help="prompt length of the prefill line (0: skip it)")
     ap.add_argument("--no-slots", action="store_true",
                     help="skip the serving path (decode and flush through a slot list)")
     ap.add_argument("--cpu-seconds", type=float, default=10.0)
@@ -611,6 +613,47 @@ def main_ours(args):
             "achieved_gbs": mb / (dm_ms / 1e3) / 1e9, "frac": mb / (dm_ms / 1e3) / 1e9 / hbm,
             "flush_avg_launch_us": fm / (km * L) * 1e3}
         del armm
+        torch.cuda.empty_cache()
+
+    # ---- prompt handoff: the FP32 recurrence over a prompt, then compression
+    if args.prefill_tokens > 0:
+        Tp = args.prefill_tokens
+        pin = I.InputStream(wl, stream=100)
+        pst = pin.state()
+        ptok = pin.tokens(Tp)
+        pdev = I.to_device(wl, {**pst, **ptok})
+        prompt = [pdev[n].transpose(0, 1).contiguous() for n in ("q", "k", "v", "beta", "decay")]
+        del pdev
+        S0p = torch.from_numpy(pst["S0"]).cuda()
+        stp = B.LQState(B.config_for(wl))
+        for _ in range(2):  # warm-up
+            stp.prefill(Tp, *prompt, S0=S0p)
+        torch.cuda.synchronize()
+        kp = 3
+        E = torch.cuda.Event
+        a, b = E(enable_timing=True), E(enable_timing=True)
+        if world > 1:
+            dist.barrier()
+        torch.cuda.synchronize()
+        a.record()
+        for _ in range(kp):
+            stp.prefill(Tp, *prompt, S0=S0p)
+        b.record()
+        torch.cuda.synchronize()
+        pms = max_over_ranks([a.elapsed_time(b)], torch, dist, world, "cuda")[0] / kp
+        status = stp.check()
+        if status != 0:
+            raise RuntimeError(f"device status after prefill: {B.STATUS_NAMES[status]}")
+        # FP32 work per head-token: decay (1), S'^T k and S'^T q (2 x 2), update (2) flops per entry
+        flops = 7.0 * wl.dk * wl.dv * nh * Tp
+        sms = props.multi_processor_count
+        alu_peak = sms * 128 * 2 * (clk["sm_max_mhz"] if clk and clk.get("sm_max_mhz") else 1965.0) * 1e6 / 1e12
+        line["prefill"] = {
+            "prompt_tokens": Tp, "value": whole_job_rate(nh * Tp, world, pms), "unit": "head-tokens/s",
+            "ms_per_launch": pms, "bound": "alu", "achieved_tflops": flops / (pms / 1e3) / 1e12,
+            "peak_tflops": alu_peak, "frac": flops / (pms / 1e3) / 1e12 / alu_peak,
+            "peak_source": f"{sms} SMs x 128 FP32 lanes x 2 flops x max SM clock"}
+        del stp, prompt
         torch.cuda.empty_cache()
 
     # ---- the serving path: the same work through a slot list

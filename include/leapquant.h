@@ -206,6 +206,28 @@ LQ_API lq_status lq_decode_steps(const lq_config *cfg, void *state, int tokens, 
                                  const void *k, const void *v, const float *beta, const float *decay,
                                  float *out, lq_stream_t stream);
 
+/* Enter a prompt: for every (slot, head), run the delta rule in FP32 over its
+ * prompt from S0 (or from a zero state), then compress the final state into
+ * a fresh blob (count 0, g 1, status cleared) as lq_state_init does with S0.
+ * The FP32 state stays on chip between the last token and the compression.
+ * Source: the state a prefill leaves enters the quantized cache (news post,
+ * per-window paragraph); the step is the delta rule of lq_decode_step.
+ *   tokens   T >= 0 (T = 0: lq_state_init from S0, or from zeros)
+ *   lengths  [N] int32, device, or NULL: row n's prompt is its first
+ *            clamp(lengths[n], 0, T) tokens; later tokens are ignored
+ *   S0       [N, H, dk, dv] f32 or NULL (zero state)
+ *   q, k     [N, T, H, dk] in_dtype     v [N, T, H, dv] in_dtype
+ *   beta     [N, T, H] f32;  decay [N, T, H] (GDN) or [N, T, H, dk] (KDA)
+ *   out      [N, T, H, dv] f32 or NULL: o_t = S_t^T q_t, zero past a row's
+ *            length
+ *   S_final  [N, H, dk, dv] f32 or NULL: the FP32 state that was compressed
+ * bits 8/6/4 only (others: LQ_ERR_UNSUPPORTED).  Alignment: S0, S_final 16
+ * bytes, lengths 4, the rest as lq_decode_step. */
+LQ_API lq_status lq_prefill(const lq_config *cfg, void *state, int tokens, const int32_t *lengths,
+                            const float *S0, const void *q, const void *k, const void *v,
+                            const float *beta, const float *decay, float *out, float *S_final,
+                            lq_stream_t stream);
+
 /* ---- Serving: a subset of the sequences through a slot list ----------
  * A continuous-batching server keeps N sequence slots in one state buffer
  * and decodes, at each step, only the sequences that are running.  The
@@ -241,6 +263,14 @@ LQ_API lq_status lq_decode_steps_slots(const lq_config *cfg, void *state, const 
                                        int n_active, int tokens, const void *q, const void *k,
                                        const void *v, const float *beta, const float *decay,
                                        float *out, lq_stream_t stream);
+
+/* lq_prefill into the slots in `slots` (row n of S0, q, k, v, beta, decay,
+ * lengths, out and S_final belongs to slot slots[n]): new requests enter
+ * free slots while the others keep decoding. */
+LQ_API lq_status lq_prefill_slots(const lq_config *cfg, void *state, const int32_t *slots,
+                                  int n_active, int tokens, const int32_t *lengths, const float *S0,
+                                  const void *q, const void *k, const void *v, const float *beta,
+                                  const float *decay, float *out, float *S_final, lq_stream_t stream);
 
 /* lq_window_flush for the slots in `slots` (slots reach their window
  * boundary at different steps when sequences join at different times). */

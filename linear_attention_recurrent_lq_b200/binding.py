@@ -21,7 +21,8 @@ STATUS_NAMES = {0: "LQ_OK", 1: "LQ_ERR_INVALID_ARG", 2: "LQ_ERR_UNSUPPORTED", 3:
 (LQ_ERR_INVALID_ARG, LQ_ERR_UNSUPPORTED, LQ_ERR_CUDA, LQ_ERR_WINDOW_FULL, LQ_ERR_RANGE,
  LQ_ERR_MISALIGNED, LQ_ERR_TIMEOUT, LQ_ERR_CORRUPT) = range(1, 9)
 ENTRY_POINTS = ("lq_validate_config", "lq_state_bytes", "lq_state_init", "lq_decode_step",
-                "lq_window_flush", "lq_dequant_state", "lq_check_status", "lq_decode_steps",
+                "lq_window_flush", "lq_dequant_state", "lq_check_status", "lq_decode_steps", "lq_prefill",
+                "lq_prefill_slots",
                 "lq_state_init_slots", "lq_decode_steps_slots",
                 "lq_decode_step_slots", "lq_window_flush_slots", "lq_copy_slots", "lq_status_string")
 
@@ -92,6 +93,10 @@ def _load():
     L.lq_decode_steps.restype = st
     L.lq_decode_steps_slots.argtypes = [P, vp, vp, i32, i32, vp, vp, vp, vp, vp, vp, vp]
     L.lq_decode_steps_slots.restype = st
+    L.lq_prefill.argtypes = [P, vp, i32, vp, vp, vp, vp, vp, vp, vp, vp, vp, vp]
+    L.lq_prefill.restype = st
+    L.lq_prefill_slots.argtypes = [P, vp, vp, i32, i32, vp, vp, vp, vp, vp, vp, vp, vp, vp, vp]
+    L.lq_prefill_slots.restype = st
     L.lq_copy_slots.restype = st
     L.lq_status_string.argtypes = [st]
     L.lq_status_string.restype = ctypes.c_char_p
@@ -193,6 +198,21 @@ def lq_decode_steps_slots(cfg, state, slots, tokens, q, k, v, beta, decay, out, 
                                      _stream(stream)), "lq_decode_steps_slots")
 
 
+def lq_prefill(cfg, state, tokens, q, k, v, beta, decay, S0=None, lengths=None, out=None, S_final=None,
+               stream=None):
+    _check(lib.lq_prefill(ctypes.byref(cfg), _ptr(state), int(tokens), _ptr(lengths), _ptr(S0), _ptr(q),
+                          _ptr(k), _ptr(v), _ptr(beta), _ptr(decay), _ptr(out), _ptr(S_final),
+                          _stream(stream)), "lq_prefill")
+
+
+def lq_prefill_slots(cfg, state, slots, tokens, q, k, v, beta, decay, S0=None, lengths=None, out=None,
+                     S_final=None, stream=None):
+    _check(lib.lq_prefill_slots(ctypes.byref(cfg), _ptr(state), _ptr(slots), _n(slots), int(tokens),
+                                _ptr(lengths), _ptr(S0), _ptr(q), _ptr(k), _ptr(v), _ptr(beta),
+                                _ptr(decay), _ptr(out), _ptr(S_final), _stream(stream)),
+           "lq_prefill_slots")
+
+
 def lq_window_flush_slots(cfg, state, slots, stream=None):
     _check(lib.lq_window_flush_slots(ctypes.byref(cfg), _ptr(state), _ptr(slots), _n(slots),
                                      _stream(stream)), "lq_window_flush_slots")
@@ -232,6 +252,11 @@ class LQState:
 
     def flush(self, stream=None):
         lq_window_flush(self.cfg, self.buf, stream)
+
+    def prefill(self, tokens, q, k, v, beta, decay, S0=None, lengths=None, out=None, S_final=None,
+                stream=None):
+        """Prompt of T tokens per (slot, head) (inputs [N, T, H, .]), then compress."""
+        lq_prefill(self.cfg, self.buf, tokens, q, k, v, beta, decay, S0, lengths, out, S_final, stream)
 
     def steps(self, tokens, q, k, v, beta, decay, out, stream=None):
         """T tokens per (slot, head): inputs [N, T, H, .], out [N, T, H, dv]."""

@@ -13,6 +13,7 @@
 #include "lq_flush.cuh"
 #include "lq_fp32.cuh"
 #include "lq_perstep.cuh"
+#include "lq_prefill.cuh"
 
 using namespace lq;
 
@@ -220,6 +221,42 @@ lq_status check_slots(const lq_config *cfg, const void *state, const int32_t *sl
     if ((int64_t)n_active * cfg->num_heads > 0x7FFFFFFF) return LQ_ERR_UNSUPPORTED;
     if (!aligned(state, 256) || !aligned(slots, 4)) return LQ_ERR_MISALIGNED;
     return LQ_OK;
+}
+
+template <int D, int BITS>
+lq_status launch_prefill(const PrefillArgs &a, cudaStream_t s) {
+    const uint32_t smem = prefill_smem_bytes(D, BITS, a.F);
+    auto k = a.map.slots ? prefill_kernel<D, BITS, true> : prefill_kernel<D, BITS, false>;
+    if (allow_smem(k, smem) != cudaSuccess) return LQ_ERR_CUDA;
+    return launched(launch_pdl(k, a.num_heads, kGroup, smem, s, a));
+}
+
+lq_status prefill_rows(const lq_config *cfg, void *state, const int32_t *slots, int rows, int tokens,
+                       const int32_t *lengths, const float *S0, const void *q, const void *k, const void *v,
+                       const float *beta, const float *decay, float *out, float *S_final, lq_stream_t stream) {
+    const lq_config &c = *cfg;
+    if (tokens < 0) return LQ_ERR_INVALID_ARG;
+    if (c.bits == 32 || c.per_step) return LQ_ERR_UNSUPPORTED;
+    if ((int64_t)rows * (tokens > 0 ? tokens : 1) * c.num_heads > 0x7FFFFFFF) return LQ_ERR_UNSUPPORTED;
+    if (rows > 0 && tokens > 0 && (!q || !k || !v || !beta || !decay)) return LQ_ERR_INVALID_ARG;
+    if (!aligned(q, 16) || !aligned(k, 16) || !aligned(v, 16) || !aligned(beta, 4) ||
+        !aligned(decay, c.decay_kind ? 16 : 4) || !aligned(out, 4) || !aligned(S0, 16) ||
+        !aligned(S_final, 16) || !aligned(lengths, 4))
+        return LQ_ERR_MISALIGNED;
+    if (rows == 0) return LQ_OK;
+    PrefillArgs a{static_cast<uint8_t *>(state), make_layout(c), make_flags(c), S0, q, k, v, beta, decay,
+                  lengths, tokens > 0 ? out : nullptr, S_final, tokens, rows * c.num_heads,
+                  SlotMap{slots, c.num_heads, c.num_slots}};
+    cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
+    switch (c.dk * 100 + c.bits) {
+        case 12808: return launch_prefill<128, 8>(a, s);
+        case 12806: return launch_prefill<128, 6>(a, s);
+        case 12804: return launch_prefill<128, 4>(a, s);
+        case 6408: return launch_prefill<64, 8>(a, s);
+        case 6406: return launch_prefill<64, 6>(a, s);
+        case 6404: return launch_prefill<64, 4>(a, s);
+        default: return LQ_ERR_UNSUPPORTED;
+    }
 }
 
 template <int MODE>
@@ -457,6 +494,27 @@ lq_status lq_copy_slots(const lq_config *cfg, void *dst, int dst_num_slots, cons
         static_cast<uint8_t *>(dst), dst_num_slots, dst_slots, static_cast<const uint8_t *>(src), src_num_slots,
         src_slots, cfg->num_heads, blob);
     return launched(cudaSuccess);
+}
+
+lq_status lq_prefill(const lq_config *cfg, void *state, int tokens, const int32_t *lengths, const float *S0,
+                     const void *q, const void *k, const void *v, const float *beta, const float *decay,
+                     float *out, float *S_final, lq_stream_t stream) {
+    lq_status st = check_config(cfg);
+    if (st != LQ_OK) return st;
+    if (!state) return LQ_ERR_INVALID_ARG;
+    if (!aligned(state, 256)) return LQ_ERR_MISALIGNED;
+    return prefill_rows(cfg, state, nullptr, cfg->num_slots, tokens, lengths, S0, q, k, v, beta, decay, out,
+                        S_final, stream);
+}
+
+lq_status lq_prefill_slots(const lq_config *cfg, void *state, const int32_t *slots, int n_active, int tokens,
+                           const int32_t *lengths, const float *S0, const void *q, const void *k, const void *v,
+                           const float *beta, const float *decay, float *out, float *S_final,
+                           lq_stream_t stream) {
+    lq_status st = check_slots(cfg, state, slots, n_active);
+    if (st != LQ_OK) return st;
+    return prefill_rows(cfg, state, slots, n_active, tokens, lengths, S0, q, k, v, beta, decay, out, S_final,
+                        stream);
 }
 
 const char *lq_status_string(lq_status s) {

@@ -154,3 +154,21 @@ def test_multi_token_arguments_rejected_before_launch(B):
     assert L.lq_decode_steps_slots(c, 256, 64, 0, 2, None, None, None, None, None, None, None) == 0
     assert L.lq_decode_steps_slots(c, 256, None, 2, 2, *ok, None) == 1
     assert L.lq_decode_steps_slots(c, 256, 64, 2, 9, *ok, None) == 2
+
+
+def test_prefill_arguments_rejected_before_launch(B):
+    cfg = B.make_config(4, 4)
+    L = B.lib
+    c = ctypes.byref(cfg)
+    inp = (16, 16, 16, 16, 16)  # q, k, v, beta, decay
+    assert L.lq_prefill(c, 256, -1, None, None, *inp, None, None, None) == 1
+    assert L.lq_prefill(c, None, 4, None, None, *inp, None, None, None) == 1
+    assert L.lq_prefill(c, 256, 4, None, None, 16, None, 16, 16, 16, None, None, None) == 1
+    assert L.lq_prefill(c, 128, 4, None, None, *inp, None, None, None) == 6
+    assert L.lq_prefill(c, 256, 4, 2, None, *inp, None, None, None) == 6      # lengths 4 B
+    assert L.lq_prefill(c, 256, 4, None, 8, *inp, None, None, None) == 6      # S0 16 B
+    assert L.lq_prefill(c, 256, 4, None, None, *inp, None, 8, None) == 6      # S_final 16 B
+    for other in (B.make_config(4, 4, bits=32), B.make_config(4, 4, bits=8, per_step=True)):
+        assert L.lq_prefill(ctypes.byref(other), 256, 4, None, None, *inp, None, None, None) == 2
+    assert L.lq_prefill_slots(c, 256, 64, 0, 4, None, None, *inp, None, None, None) == 0
+    assert L.lq_prefill_slots(c, 256, None, 2, 4, None, None, *inp, None, None, None) == 1
