@@ -27,7 +27,7 @@
  *    except lq_check_status, which synchronizes the stream.
  *  - Argument errors are reported before anything is launched (LQ_ERR_*).
  *    A failed launch returns LQ_ERR_CUDA.  Conditions that depend on data on
- *    the device (a full window, a decay product out of range, a timed-out
+ *    the device (a full window, a negative or NaN gate, a timed-out
  *    wait) set a sticky bit in that (slot, head)'s status word; the kernels
  *    then skip that (slot, head) and never trap.  lq_check_status reads them.
  *  - Tensors are dense, row-major, contiguous.  N = num_slots (sequences),
@@ -107,7 +107,7 @@ typedef enum lq_status {
     LQ_ERR_UNSUPPORTED = 2,  /* valid but not built: see lq_validate_config   */
     LQ_ERR_CUDA = 3,         /* a CUDA call or launch failed                  */
     LQ_ERR_WINDOW_FULL = 4,  /* device: decode step into a window of W pairs  */
-    LQ_ERR_RANGE = 5,        /* device: decay product left [2^-96, 1]         */
+    LQ_ERR_RANGE = 5,        /* device: a gate (decay) was negative or NaN    */
     LQ_ERR_MISALIGNED = 6,   /* a pointer breaks the alignment rule above     */
     LQ_ERR_TIMEOUT = 7,      /* device: an on-chip copy wait gave up          */
     LQ_ERR_CORRUPT = 8       /* device: a blob header failed its checks       */
@@ -163,7 +163,15 @@ LQ_API lq_status lq_state_init(const lq_config *cfg, void *state, const float *S
  * buffered pairs (abstract; per-window paragraph).  A (slot, head) whose
  * window already holds W pairs, or whose status is nonzero, is skipped: its
  * output row is written as zeros and its state is left unchanged.  Call
- * lq_window_flush after every W steps. */
+ * lq_window_flush after every W steps.
+ * Gates may be as small as 0.  The buffered keys are stored divided by the
+ * decay product since the window start; when a key channel's product falls
+ * below 2^-96 the step first moves the window frame to the current token:
+ * that channel's factor is multiplied into its smoothing scale (rounded to
+ * the scale's storage type), its compensator entries and the buffered keys,
+ * and its product restarts at 1 (the state stands for the same matrix, up to
+ * one rounding per stored value).  A negative or NaN gate sets LQ_DEV_RANGE
+ * and skips the (slot, head). */
 LQ_API lq_status lq_decode_step(const lq_config *cfg, void *state, const void *q, const void *k,
                          const void *v, const float *beta, const float *decay, float *out,
                          lq_stream_t stream);

@@ -524,7 +524,7 @@ const char *lq_status_string(lq_status s) {
         case LQ_ERR_UNSUPPORTED: return "configuration not supported by this build";
         case LQ_ERR_CUDA: return "CUDA error";
         case LQ_ERR_WINDOW_FULL: return "decode step into a full window (flush every W steps)";
-        case LQ_ERR_RANGE: return "window decay product fell below 2^-96";
+        case LQ_ERR_RANGE: return "a gate (decay) was negative or NaN";
         case LQ_ERR_MISALIGNED: return "pointer misaligned (see the alignment rule in leapquant.h)";
         case LQ_ERR_TIMEOUT: return "on-chip copy wait timed out";
         case LQ_ERR_CORRUPT: return "state blob header failed its checks";

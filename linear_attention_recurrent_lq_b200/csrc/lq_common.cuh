@@ -18,7 +18,8 @@ constexpr int kMaxComp = 16;
 constexpr int kMaxWindow = 64;
 // Decay products below this leave the window-start frame's safe range: the
 // keys are stored divided by the product, so it must stay far from FP32
-// underflow.
+// underflow.  The decode moves the frame (rebase_frame) when a product
+// falls below it.
 constexpr float kMinDecayProduct = 0x1p-96f;
 // Bounded waits on on-chip copies: give up after this long (ns).
 constexpr unsigned long long kWaitLimitNs = 1000000000ull;

@@ -78,6 +78,74 @@ __host__ __device__ inline DecodeStage decode_stage(const Layout &L, int D, int 
 // (two of them, by head parity):
 //   y [2D] f32 | X [2D] int16 | chunk scales [2*D/16] | khat [D] | g [D]
 //   | column terms float2 [D] | row / column compensator lists [2*16] | info [8]
+// Move the window frame of one head to the current token.  Within a window
+// the state is diag(g)(S_base + sum_m khat_m u_m^T); when the decay product
+// g_i of key channel i falls below kMinDecayProduct, channel i's factor
+// f_i = g_i goes into what is stored instead: the smoothing scale sm_i (the
+// base row i, rounded to the scale's storage format), the compensator
+// entries of row i, and khat_m[i] of every buffered pair; g_i restarts at 1.
+// Exact algebra up to one rounding per stored value; the base part taken
+// along is below 2^-96 of its size at the window start.  Runs in the prep
+// warp: lane l scales keys KPL*l .., f[e] its factors (1: channel kept).  The
+// stage and the blob get the same values.
+template <int D>
+__device__ __noinline__ void rebase_frame(uint8_t *st, uint8_t *blob, const Layout &L, uint32_t pairs_at,
+                                          uint32_t count, uint32_t ncomp, int f16, const float (&f)[D / 32],
+                                          int lane) {
+    constexpr int KPL = D / 32;
+    const int i0 = KPL * lane;
+#pragma unroll
+    for (int e = 0; e < KPL; ++e) {
+        const int i = i0 + e;
+        const float v = load_scale(st + L.sm_off, i, f16) * f[e];
+        if (f16) {
+            const __half hv = __float2half_rn(v);
+            reinterpret_cast<__half *>(st + L.sm_off)[i] = hv;
+            reinterpret_cast<__half *>(blob + L.sm_off)[i] = hv;
+        } else {
+            reinterpret_cast<float *>(st + L.sm_off)[i] = v;
+            reinterpret_cast<float *>(blob + L.sm_off)[i] = v;
+        }
+    }
+    for (uint32_t m = 0; m < count; ++m) {
+        float *ks = reinterpret_cast<float *>(st + pairs_at + (size_t)m * L.pair_bytes);
+        float *kb = reinterpret_cast<float *>(blob + L.pairs_off + (size_t)m * L.pair_bytes);
+#pragma unroll
+        for (int e = 0; e < KPL; ++e) {
+            const float v = ks[i0 + e] * f[e];
+            ks[i0 + e] = v;
+            kb[i0 + e] = v;
+        }
+    }
+    const uint32_t *meta = reinterpret_cast<const uint32_t *>(st + kHdrMeta);
+    for (uint32_t c = 0; c < ncomp && c < (uint32_t)kMaxComp; ++c) {
+        float *vs = reinterpret_cast<float *>(st + L.cvec_off) + (size_t)c * D;
+        float *vb = reinterpret_cast<float *>(blob + L.cvec_off) + (size_t)c * D;
+        const uint32_t m = meta[c];
+        if (m & kCompCol) {  // a value column over the keys: entry i takes f_i
+#pragma unroll
+            for (int e = 0; e < KPL; ++e) {
+                const float v = vs[i0 + e] * f[e];
+                vs[i0 + e] = v;
+                vb[i0 + e] = v;
+            }
+        } else {  // key row r over the values: every entry takes f_r
+            const int r = (int)(m & 0x7FFFFFFFu) % D;
+            float fr = 1.f;
+#pragma unroll
+            for (int e = 0; e < KPL; ++e)
+                if (r % KPL == e) fr = f[e];
+            fr = __shfl_sync(0xFFFFFFFFu, fr, r / KPL);
+            for (int j = lane; j < D; j += 32) {
+                const float v = vs[j] * fr;
+                vs[j] = v;
+                vb[j] = v;
+            }
+        }
+    }
+    __syncwarp();
+}
+
 template <int D>
 struct PrepBuf {
     static constexpr uint32_t y = 0, X = 8 * D, sc = 12 * D, kh = sc + 8 * (D / 16), g = kh + 4 * D,
@@ -465,6 +533,37 @@ __global__ void __launch_bounds__(D + 64, (SLOTS || MULTI) ? 3 : 0) decode_kerne
 #pragma unroll
                     for (int e = 0; e < KPL; ++e) gn[e] = gprev[e] * alpha;
                 }
+                // A decay product below the window frame's range moves the frame
+                // (rebase_frame): the stored parts take the factor and the
+                // product of those channels restarts at 1.  A negative or NaN
+                // gate is an input error (RANGE below).
+                bool small = false, invalid = false, rebase_timeout = false;
+#pragma unroll
+                for (int e = 0; e < KPL; ++e) {
+                    invalid |= !(gn[e] >= 0.f);
+                    small |= gn[e] < kMinDecayProduct;
+                }
+                if (__any_sync(0xFFFFFFFFu, small) && !__any_sync(0xFFFFFFFFu, invalid)) {
+                    // inside one head, the consumers must be done with the previous
+                    // token (its pair is in the stage and the blob) first
+                    const bool waited = !(MULTI && t > 0) ||
+                                        mbar_wait_bounded(&pempty[(step - 1) & 1], (uint32_t)((step - 1) >> 1) & 1u);
+                    if (waited) {
+                        float f[KPL];
+#pragma unroll
+                        for (int e = 0; e < KPL; ++e) f[e] = (!F.kda || gn[e] < kMinDecayProduct) ? gn[e] : 1.f;
+                        const int bh = blob_of(A.map, (int)(blockIdx.x + (size_t)it * G));
+                        rebase_frame<D>(const_cast<uint8_t *>(st), A.state + (size_t)bh * L.blob, L, SG.pairs_at,
+                                        hdr.x + (uint32_t)t, hdr.z, F.f16_scale, f, lane);
+#pragma unroll
+                        for (int e = 0; e < KPL; ++e)
+                            if (!F.kda || gn[e] < kMinDecayProduct) gn[e] = 1.f;
+                    } else {
+                        if (lane == 0) *s_abort = 1u;
+                        rebase_timeout = true;  // the head is skipped below
+                        gn[0] = __int_as_float(0x7FC00000);
+                    }
+                }
 #pragma unroll
                 for (int e = 0; e < KPL; ++e) gprev[e] = gn[e];
                 bool bad = false;
@@ -535,7 +634,7 @@ __global__ void __launch_bounds__(D + 64, (SLOTS || MULTI) ? 3 : 0) decode_kerne
                 if (bad) {
                     run = false;
                     dead = true;  // the later tokens of this head are skipped too
-                    newbits = LQ_DEV_RANGE;
+                    newbits = rebase_timeout ? LQ_DEV_TIMEOUT : LQ_DEV_RANGE;
                 }
             }
             if (lane == 0) {

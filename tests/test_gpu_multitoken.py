@@ -138,15 +138,15 @@ def test_window_without_room_skips_the_whole_head():
     assert torch.equal(v[:, :4], bv[:, :4]) and torch.equal(v[:, 8:], bv[:, 8:])
 
 
-def test_range_failure_mid_call_keeps_the_earlier_tokens():
-    """GDN decay 2^-40 per token: the decay product leaves the range at the
-    third token.  Tokens 0 and 1 commit; the rest of the head is skipped,
-    exactly as single-token calls behave."""
+def test_invalid_gate_mid_call_keeps_the_earlier_tokens():
+    """A NaN gate at the third token of a head: tokens 0 and 1 commit; the
+    rest of that head is skipped with the RANGE bit, exactly as single-token
+    calls behave."""
     wl, bits = CASES["gdn_int8"]
     Wn, T = 8, 5
     d = I.draw(wl, T)
     dev = device_inputs(wl, d)
-    dev["decay"] = torch.full_like(dev["decay"], 2.0 ** -40)
+    dev["decay"][2, 1, 2] = float("nan")  # token 2, row 1, head 2
     a, b = _state(wl, bits, Wn), _state(wl, bits, Wn)
     S0 = torch.from_numpy(d["S0"]).cuda()
     a.init(S0)
@@ -158,7 +158,8 @@ def test_range_failure_mid_call_keeps_the_earlier_tokens():
     torch.cuda.synchronize()
     assert torch.equal(out, ref.transpose(0, 1))
     assert torch.equal(a.buf, b.buf)
-    assert out[:, :2].abs().sum() > 0 and not out[:, 2:].any()
+    assert out[1, :2, 2].abs().sum() > 0 and not out[1, 2:, 2].any()
+    assert out[0].abs().sum() > 0
     from linear_attention_recurrent_lq_b200 import binding as B
     assert b.check() == B.LQ_ERR_RANGE
 

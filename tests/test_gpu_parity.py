@@ -317,7 +317,10 @@ def test_step_into_full_window_is_flagged_and_skipped():
     assert changed[:, :4].sum() == 0 and changed[:, 8:].sum() == 0
 
 
-def test_decay_underflow_is_flagged():
+def test_decay_underflow_moves_the_window_frame():
+    """Gates of 2^-40: the third token takes the decay product below 2^-96,
+    so the frame moves to it (no status bit, the stored product restarts at
+    1).  A zero gate then forgets everything: the state is beta k v^T."""
     from linear_attention_recurrent_lq_b200 import binding as B
     wl = SMALL["gdn_int8"].replace(window=8)
     d = I.draw(wl, 4)
@@ -327,11 +330,20 @@ def test_decay_underflow_is_flagged():
     dev = device_inputs(wl, d)
     out = torch.empty((wl.batch, wl.heads, wl.dv), device="cuda")
     tiny = torch.full_like(dev["decay"][0], 2.0 ** -40)
-    st.step(dev["q"][0], dev["k"][0], dev["v"][0], dev["beta"][0], tiny, out)
-    st.step(dev["q"][1], dev["k"][1], dev["v"][1], dev["beta"][1], tiny, out)
+    for t in range(3):  # 2^-40, 2^-80, then 2^-120 < 2^-96
+        st.step(dev["q"][t], dev["k"][t], dev["v"][t], dev["beta"][t], tiny, out)
     assert st.check() == 0
-    st.step(dev["q"][2], dev["k"][2], dev["v"][2], dev["beta"][2], tiny, out)  # 2^-120 < 2^-96
-    assert st.check() == 5  # LQ_ERR_RANGE
+    g = st.blobs().cpu().numpy()[:, 16:20].copy().view(np.float32)[:, 0]
+    np.testing.assert_array_equal(g, np.ones_like(g))
+    st.step(dev["q"][3], dev["k"][3], dev["v"][3], dev["beta"][3], torch.zeros_like(tiny), out)
+    assert st.check() == 0
+    S = st.dequant().cpu().numpy().reshape(-1, wl.dk, wl.dv)
+    nh = wl.batch * wl.heads
+    k = d["k"][3].reshape(nh, wl.dk).astype(np.float64)
+    v = d["v"][3].reshape(nh, wl.dv).astype(np.float64)
+    beta = d["beta"][3].reshape(nh).astype(np.float64)
+    for h in range(nh):
+        np.testing.assert_allclose(S[h], beta[h] * np.outer(k[h], v[h]), rtol=1e-6, atol=1e-30)
 
 
 def test_snapshot_restore_continues_bitwise():
