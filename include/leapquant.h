@@ -298,6 +298,14 @@ LQ_API lq_status lq_copy_slots(const lq_config *cfg, void *dst, int dst_num_slot
                                const int32_t *dst_slots, const void *src, int src_num_slots,
                                const int32_t *src_slots, int n, lq_stream_t stream);
 
+/* Diagnostic of the device-side failure detection: one kernel thread waits,
+ * through the bounded wait every kernel of this library uses, on an on-chip
+ * barrier that nothing ever arrives on.  The wait gives up after its time
+ * limit (one second) and the kernel writes LQ_DEV_TIMEOUT to *status (a
+ * device uint32, 4-byte aligned), then exits: the context stays usable.
+ * Enqueued on `stream`; the call does not wait. */
+LQ_API lq_status lq_selftest_wait(uint32_t *status, lq_stream_t stream);
+
 /* Static text for a status code. */
 LQ_API const char *lq_status_string(lq_status s);
 

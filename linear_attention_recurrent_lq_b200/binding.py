@@ -21,10 +21,10 @@ STATUS_NAMES = {0: "LQ_OK", 1: "LQ_ERR_INVALID_ARG", 2: "LQ_ERR_UNSUPPORTED", 3:
 (LQ_ERR_INVALID_ARG, LQ_ERR_UNSUPPORTED, LQ_ERR_CUDA, LQ_ERR_WINDOW_FULL, LQ_ERR_RANGE,
  LQ_ERR_MISALIGNED, LQ_ERR_TIMEOUT, LQ_ERR_CORRUPT) = range(1, 9)
 ENTRY_POINTS = ("lq_validate_config", "lq_state_bytes", "lq_state_init", "lq_decode_step",
-                "lq_window_flush", "lq_dequant_state", "lq_check_status", "lq_decode_steps", "lq_prefill",
-                "lq_prefill_slots",
-                "lq_state_init_slots", "lq_decode_steps_slots",
-                "lq_decode_step_slots", "lq_window_flush_slots", "lq_copy_slots", "lq_status_string")
+                "lq_decode_steps", "lq_window_flush", "lq_dequant_state", "lq_check_status",
+                "lq_prefill", "lq_state_init_slots", "lq_decode_step_slots", "lq_decode_steps_slots",
+                "lq_window_flush_slots", "lq_prefill_slots", "lq_copy_slots", "lq_selftest_wait",
+                "lq_status_string")
 
 
 class LQError(RuntimeError):
@@ -98,6 +98,8 @@ def _load():
     L.lq_prefill_slots.argtypes = [P, vp, vp, i32, i32, vp, vp, vp, vp, vp, vp, vp, vp, vp, vp]
     L.lq_prefill_slots.restype = st
     L.lq_copy_slots.restype = st
+    L.lq_selftest_wait.argtypes = [vp, vp]
+    L.lq_selftest_wait.restype = st
     L.lq_status_string.argtypes = [st]
     L.lq_status_string.restype = ctypes.c_char_p
     return L
@@ -224,6 +226,11 @@ def lq_copy_slots(cfg, dst, dst_num_slots, dst_slots, src, src_num_slots, src_sl
     _check(lib.lq_copy_slots(ctypes.byref(cfg), _ptr(dst), int(dst_num_slots), _ptr(dst_slots),
                              _ptr(src), int(src_num_slots), _ptr(src_slots), _n(src_slots),
                              _stream(stream)), "lq_copy_slots")
+
+
+def lq_selftest_wait(status, stream=None):
+    """Device diagnostic: a bounded wait that runs out writes LQ_DEV_TIMEOUT to status."""
+    _check(lib.lq_selftest_wait(_ptr(status), _stream(stream)), "lq_selftest_wait")
 
 
 class LQState:

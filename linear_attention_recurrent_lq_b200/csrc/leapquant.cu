@@ -212,6 +212,17 @@ __global__ void __launch_bounds__(256) copy_slots_kernel(uint8_t *dst, int dst_s
     for (uint32_t x = threadIdx.x; x < blob / 16u; x += 256u) to[x] = __ldg(from + x);
 }
 
+// Diagnostic: one thread waits, through the same bounded wait every kernel
+// uses, on a barrier that nothing arrives on; when the wait gives up it
+// records LQ_DEV_TIMEOUT in *status (0 if the wait ever succeeded).
+__global__ void selftest_wait_kernel(uint32_t *status) {
+    __shared__ __align__(8) uint64_t bar;
+    if (threadIdx.x != 0) return;
+    mbar_init(&bar, 1);
+    fence_mbar_init();
+    *status = mbar_wait_bounded(&bar, 0u) ? 0u : LQ_DEV_TIMEOUT;
+}
+
 // Checks shared by the entry points that take a slot list.
 lq_status check_slots(const lq_config *cfg, const void *state, const int32_t *slots, int n_active) {
     lq_status st = check_config(cfg);
@@ -515,6 +526,13 @@ lq_status lq_prefill_slots(const lq_config *cfg, void *state, const int32_t *slo
     if (st != LQ_OK) return st;
     return prefill_rows(cfg, state, slots, n_active, tokens, lengths, S0, q, k, v, beta, decay, out, S_final,
                         stream);
+}
+
+lq_status lq_selftest_wait(uint32_t *status, lq_stream_t stream) {
+    if (!status) return LQ_ERR_INVALID_ARG;
+    if (!aligned(status, 4)) return LQ_ERR_MISALIGNED;
+    selftest_wait_kernel<<<1, 32, 0, reinterpret_cast<cudaStream_t>(stream)>>>(status);
+    return launched(cudaSuccess);
 }
 
 const char *lq_status_string(lq_status s) {

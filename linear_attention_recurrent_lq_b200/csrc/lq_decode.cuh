@@ -376,14 +376,12 @@ __global__ void __launch_bounds__(D + 64, (SLOTS || MULTI) ? 3 : 0) decode_kerne
     __syncthreads();
     // While the previous kernel on the stream drains, start pulling this
     // CTA's first two blobs (compact state and codes) into L2.  A prefetch
-    // changes no data, so it is safe whatever that kernel writes.  (A slot
-    // list read here may still be changing: a stale entry, bounds-checked
-    // like any other, only wastes the prefetch.)
-    if (tid == 0)
-        for (int it = 0; it < 2 && it < n_mine; ++it) {
-            const int b = blob_of(A.map, (int)blockIdx.x + it * G);
-            if (b >= 0) bulk_prefetch_l2(A.state + (size_t)b * L.blob, L.pairs_off);
-        }
+    // changes no data, so it is safe whatever that kernel writes.  Not
+    // through a slot list: the list would have to be read first, and that
+    // read measured slower than no prefetch at all.
+    if (tid == 0 && !SLOTS)
+        for (int it = 0; it < 2 && it < n_mine; ++it)
+            bulk_prefetch_l2(A.state + ((size_t)blockIdx.x + (size_t)it * G) * L.blob, L.pairs_off);
     pdl_wait();
     pdl_trigger();
 

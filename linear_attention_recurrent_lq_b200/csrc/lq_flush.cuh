@@ -743,8 +743,9 @@ __global__ void __launch_bounds__(kGroup, 2) flush_kernel(FlushArgs A) {
 
     // pull the first two blobs into L2 while the previous kernel drains (a
     // prefetch changes no data; a slot list read here may still be changing:
-    // a stale entry, bounds-checked like any other, only wastes the prefetch)
-    if (tid == 0)
+    // a stale entry, bounds-checked like any other, only wastes the prefetch;
+    // its read goes to a thread other than the one that stages the blobs)
+    if (tid == (SLOTS ? 32 : 0))
         for (int it = 0; it < kFlushStages && it < n_mine; ++it) {
             const uint8_t *b = blob_at(it);
             if (b) bulk_prefetch_l2(b, L.pairs_off + (uint32_t)F.window * L.pair_bytes);

@@ -172,3 +172,8 @@ def test_prefill_arguments_rejected_before_launch(B):
         assert L.lq_prefill(ctypes.byref(other), 256, 4, None, None, *inp, None, None, None) == 2
     assert L.lq_prefill_slots(c, 256, 64, 0, 4, None, None, *inp, None, None, None) == 0
     assert L.lq_prefill_slots(c, 256, None, 2, 4, None, None, *inp, None, None, None) == 1
+
+
+def test_selftest_wait_arguments(B):
+    assert B.lib.lq_selftest_wait(None, None) == 1
+    assert B.lib.lq_selftest_wait(2, None) == 6
