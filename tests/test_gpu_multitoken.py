@@ -189,3 +189,28 @@ def test_multi_token_through_a_slot_list():
         assert torch.equal(oa, of)
         for n, s in enumerate(slots):
             assert torch.equal(full.blobs()[s * H:(s + 1) * H], alone.blobs()[n * H:(n + 1) * H])
+
+
+def test_multi_token_at_the_largest_window_and_compensator_count():
+    """W = 64, r = 16, T = 8 (KDA, the largest stage): a whole window in
+    eight calls, then the flush, bitwise equal to single-token calls."""
+    wl = W["kda_int8_b128h32"].replace(batch=2, heads=2, num_comp=16)
+    bits, Wn, T = 8, 64, 8
+    d = I.draw(wl, Wn)
+    dev = device_inputs(wl, d)
+    a, b = _state(wl, bits, Wn), _state(wl, bits, Wn)
+    S0 = torch.from_numpy(d["S0"]).cuda()
+    a.init(S0)
+    b.init(S0)
+    for t0 in range(0, Wn, T):
+        ref = torch.empty((T, wl.batch, wl.heads, wl.dv), dtype=torch.float32, device="cuda")
+        _single(a, dev, t0, T, ref)
+        out = torch.empty((wl.batch, T, wl.heads, wl.dv), dtype=torch.float32, device="cuda")
+        b.steps(T, *_stack(dev, t0, T), out)
+        torch.cuda.synchronize()
+        assert torch.equal(out, ref.transpose(0, 1)), t0
+    a.flush()
+    b.flush()
+    torch.cuda.synchronize()
+    assert torch.equal(a.buf, b.buf)
+    assert b.check() == 0
