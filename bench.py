@@ -400,20 +400,17 @@ def time_arm(arm, steps, warmup, torch, dist, world):
 
 def time_e2e(arm, host, steps, torch, dist, world):
     """Same steps through the public calls with host buffers: every step
-    copies its inputs host->device from pinned memory, runs the window and
-    copies every output back."""
-    h2d = sum(t.numel() * t.element_size() for ld in host for t in ld["in"].values())
-    d2h = sum(o.numel() * o.element_size() for o in arm.out)
-
-    def one():
-        for l, ld in enumerate(host):
-            for name, t in ld["in"].items():
-                arm.inp[l][name].copy_(t, non_blocking=True)
-        arm.step()
-        for l, ld in enumerate(host):
-            ld["out"].copy_(arm.out[l], non_blocking=True)
-
-    one()
+    copies each layer's inputs host->device from pinned memory, runs its
+    window and copies every output back, the transfers overlapped with the
+    kernels of the neighbouring layers (pipeline.HostIOPipeline)."""
+    from linear_attention_recurrent_lq_b200.pipeline import HostIOPipeline, Layer
+    layers = [Layer(arm.states[l], arm.inp[l], arm.out[l], host[l]["in"], host[l]["out"]) for l in range(arm.L)]
+    pipe = HostIOPipeline(layers, arm.wl.window, flush=arm.has_flush)
+    pipe.capture()
+    h2d, d2h = pipe.bytes_per_step()
+    pipe.fork()
+    pipe.step()
+    pipe.join()
     torch.cuda.synchronize()
     E = torch.cuda.Event
     start, end = E(enable_timing=True), E(enable_timing=True)
@@ -421,8 +418,10 @@ def time_e2e(arm, host, steps, torch, dist, world):
         dist.barrier()
     torch.cuda.synchronize()
     start.record()
+    pipe.fork()
     for _ in range(steps):
-        one()
+        pipe.step()
+    pipe.join()
     end.record()
     torch.cuda.synchronize()
     if world > 1:
