@@ -209,7 +209,10 @@ LQ_API lq_status lq_check_status(const lq_config *cfg, const void *state, lq_str
  * whole (LQ_DEV_WINDOW_FULL, zero outputs).  If token t fails its range
  * check, tokens t.. of that (slot, head) are skipped (zero outputs) and the
  * state keeps the pairs of tokens < t.  bits 8/6/4 only (others:
- * LQ_ERR_UNSUPPORTED).  T = 1 is lq_decode_step. */
+ * LQ_ERR_UNSUPPORTED).  T = 1 is lq_decode_step.  Every token is committed;
+ * to keep only an accepted prefix (speculative decoding), snapshot the rows
+ * first with lq_copy_slots, restore the rows that rejected tokens and decode
+ * their accepted prefix again. */
 LQ_API lq_status lq_decode_steps(const lq_config *cfg, void *state, int tokens, const void *q,
                                  const void *k, const void *v, const float *beta, const float *decay,
                                  float *out, lq_stream_t stream);
