@@ -128,13 +128,24 @@ def fp32_bytes(wl):
 
 # ------------------------------------------------------------ helpers
 
+def strip_comments(src: str) -> str:
+    """C/C++ source without comments and blank space: what the compiler sees
+    of it (string literals with comment markers do not occur in these files)."""
+    import re
+    src = re.sub(r"/\*.*?\*/", " ", src, flags=re.S)
+    src = re.sub(r"//[^\n]*", " ", src)
+    return " ".join(src.split())
+
+
 def kernel_source_sha():
+    """Hash of the CUDA sources and the C header, comments left out, so a
+    profile taken on the same code stays valid across comment edits."""
     h = hashlib.sha256()
     paths = sorted(os.path.join(ROOT, "linear_attention_recurrent_lq_b200", "csrc", n)
                    for n in os.listdir(os.path.join(ROOT, "linear_attention_recurrent_lq_b200", "csrc")))
     for p in paths + [os.path.join(ROOT, "include", "leapquant.h")]:
-        with open(p, "rb") as fh:
-            h.update(fh.read())
+        with open(p, encoding="utf-8") as fh:
+            h.update(strip_comments(fh.read()).encode())
     return h.hexdigest()[:16]
 
 
