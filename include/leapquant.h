@@ -157,7 +157,7 @@ LQ_API lq_status lq_state_init(const lq_config *cfg, void *state, const float *S
  *   q, k   [N, H, dk]  in_dtype  in
  *   v      [N, H, dv]  in_dtype  in
  *   beta   [N, H] f32            in, write strength
- *   decay  [N, H] f32 (GDN: alpha) or [N, H, dk] f32 (KDA: a), in (0, 1]
+ *   decay  [N, H] f32 (GDN: alpha) or [N, H, dk] f32 (KDA: a), in [0, 1]
  *   out    [N, H, dv] f32        out, o_t = S_t^T q_t
  * Outputs come from the fixed low-bit state, the compensators and the
  * buffered pairs (abstract; per-window paragraph).  A (slot, head) whose
@@ -249,10 +249,11 @@ LQ_API lq_status lq_prefill(const lq_config *cfg, void *state, int tokens, const
  *          is undefined, every access still stays inside the buffers).
  * Every kernel bounds-checks each entry against [0, N): a row whose slot is
  * out of range touches no blob; its output row (decode) is written as
- * zeros.  n_active = 0 launches nothing and returns LQ_OK.  These three take
- * the LeapQuant formats only (bits 8/6/4, per_step = 0), else
- * LQ_ERR_UNSUPPORTED.  The list is read on the device when the kernel runs,
- * so it may be written by earlier work on the same stream. */
+ * zeros.  n_active = 0 launches nothing and returns LQ_OK.  The init,
+ * decode, prefill and flush calls below take the LeapQuant formats only
+ * (bits 8/6/4, per_step = 0), else LQ_ERR_UNSUPPORTED; lq_copy_slots takes
+ * any format.  The list is read on the device when the kernel runs, so it
+ * may be written by earlier work on the same stream. */
 
 /* lq_state_init for the slots in `slots`:
  *   S0 [n_active, H, dk, dv] f32, in (row n enters slot slots[n]).
