@@ -550,7 +550,7 @@ def main_ours(args):
         "config": config_of(wl, args, world),
         "roofline": {"bound": "hbm", "achieved": achieved, "peak": hbm, "unit": "GB/s",
                      "frac": achieved / hbm, "traffic": traffic,
-                     "kernel": "decode_kernel<128,8>", "peak_source": f"{peak_kind} hbm_gbs",
+                     "kernel": f"decode_kernel<{wl.dk},{wl.bits}>", "peak_source": f"{peak_kind} hbm_gbs",
                      "algorithmic_bytes_per_launch": dec_bytes_per_launch,
                      "avg_launch_us": dec_ms * 1e3},
         "step_hbm": {"algorithmic_bytes_per_step": step_bytes,
