@@ -266,6 +266,9 @@ class Arm:
         self.bits = bits
         self.has_flush = bits != 32 and not per_step
         self.L = len(layers_data)
+        # token-major order over two or more layer-states: the launch before a
+        # decode is always another state's decode or flush
+        self.flags = B.LQ_STEP_EARLY_STATE if (self.has_flush and self.L >= 2) else 0
         self.states, self.inp, self.out = [], [], []
         for ld in layers_data:
             st = B.LQState(self.cfg)
@@ -282,7 +285,7 @@ class Arm:
             for l in range(self.L):
                 x = self.inp[l]
                 self.states[l].step(x["q"][t], x["k"][t], x["v"][t], x["beta"][t], x["decay"][t],
-                                    self.out[l][t])
+                                    self.out[l][t], flags=self.flags)
 
     def flush_all(self):
         if not self.has_flush:
@@ -495,6 +498,8 @@ def config_of(wl, args, world):
             "qkv_dtype": wl.in_dtype, "layers_rotated": args.layers,
             "step": f"one window: {wl.window} decode tokens x {args.layers} layers + {args.layers} flushes",
             "l2": "no flush: the rotated layer-states are larger than L2",
+            "decode_call": ("lq_decode_step_ex(LQ_STEP_EARLY_STATE): the launch before each decode is "
+                            "another layer-state's" if args.layers >= 2 else "lq_decode_step"),
             "parallelism": f"replicas x{world}" if world > 1 else "single GPU"}
 
 

@@ -196,6 +196,22 @@ LQ_API lq_status lq_dequant_state(const lq_config *cfg, const void *state, float
  * device pointer; the read uses one strided device-to-host copy. */
 LQ_API lq_status lq_check_status(const lq_config *cfg, const void *state, lq_stream_t stream);
 
+/* lq_decode_step with call flags:
+ *   LQ_STEP_EARLY_STATE  the kernel enqueued on `stream` just before this
+ *      call does not write `state` (it may still be running when this one
+ *      starts: the library launches with programmatic dependent launch).
+ *      The step then stages its first blobs' compact state and codes while
+ *      that kernel drains; q, k, v, beta and decay are still read only after
+ *      it has completed.  True in a model when the previous kernel is, say,
+ *      the projection that produces q, k, v; false when two steps on the same
+ *      state follow each other directly.  A wrong promise reads stale state.
+ * Other bits: LQ_ERR_INVALID_ARG.  The flag changes nothing for bits = 32
+ * and per_step states. */
+#define LQ_STEP_EARLY_STATE 0x1u
+LQ_API lq_status lq_decode_step_ex(const lq_config *cfg, void *state, const void *q, const void *k,
+                                   const void *v, const float *beta, const float *decay, float *out,
+                                   uint32_t flags, lq_stream_t stream);
+
 /* T consecutive tokens for every (slot, head) in one launch (speculative
  * verification, multi-token prediction): the compact state is read once for
  * all T tokens.  Token t's output and pair equal those of the t-th of T

@@ -20,7 +20,7 @@ STATUS_NAMES = {0: "LQ_OK", 1: "LQ_ERR_INVALID_ARG", 2: "LQ_ERR_UNSUPPORTED", 3:
                 7: "LQ_ERR_TIMEOUT", 8: "LQ_ERR_CORRUPT"}
 (LQ_ERR_INVALID_ARG, LQ_ERR_UNSUPPORTED, LQ_ERR_CUDA, LQ_ERR_WINDOW_FULL, LQ_ERR_RANGE,
  LQ_ERR_MISALIGNED, LQ_ERR_TIMEOUT, LQ_ERR_CORRUPT) = range(1, 9)
-ENTRY_POINTS = ("lq_validate_config", "lq_state_bytes", "lq_state_init", "lq_decode_step",
+ENTRY_POINTS = ("lq_validate_config", "lq_state_bytes", "lq_state_init", "lq_decode_step", "lq_decode_step_ex",
                 "lq_decode_steps", "lq_window_flush", "lq_dequant_state", "lq_check_status",
                 "lq_prefill", "lq_state_init_slots", "lq_decode_step_slots", "lq_decode_steps_slots",
                 "lq_window_flush_slots", "lq_prefill_slots", "lq_copy_slots", "lq_selftest_wait",
@@ -75,6 +75,8 @@ def _load():
     L.lq_state_init.restype = st
     L.lq_decode_step.argtypes = [P, vp, vp, vp, vp, vp, vp, vp, vp]
     L.lq_decode_step.restype = st
+    L.lq_decode_step_ex.argtypes = [P, vp, vp, vp, vp, vp, vp, vp, ctypes.c_uint32, vp]
+    L.lq_decode_step_ex.restype = st
     L.lq_window_flush.argtypes = [P, vp, vp]
     L.lq_window_flush.restype = st
     L.lq_dequant_state.argtypes = [P, vp, vp, vp]
@@ -158,6 +160,15 @@ def lq_decode_step(cfg, state, q, k, v, beta, decay, out, stream=None):
     _check(lib.lq_decode_step(ctypes.byref(cfg), _ptr(state), _ptr(q), _ptr(k), _ptr(v),
                               _ptr(beta), _ptr(decay), _ptr(out), _stream(stream)),
            "lq_decode_step")
+
+
+LQ_STEP_EARLY_STATE = 0x1
+
+
+def lq_decode_step_ex(cfg, state, q, k, v, beta, decay, out, flags=0, stream=None):
+    _check(lib.lq_decode_step_ex(ctypes.byref(cfg), _ptr(state), _ptr(q), _ptr(k), _ptr(v),
+                                 _ptr(beta), _ptr(decay), _ptr(out), int(flags), _stream(stream)),
+           "lq_decode_step_ex")
 
 
 def lq_window_flush(cfg, state, stream=None):
@@ -254,8 +265,11 @@ class LQState:
     def init(self, S0, stream=None):
         lq_state_init(self.cfg, self.buf, S0, stream)
 
-    def step(self, q, k, v, beta, decay, out, stream=None):
-        lq_decode_step(self.cfg, self.buf, q, k, v, beta, decay, out, stream)
+    def step(self, q, k, v, beta, decay, out, stream=None, flags=0):
+        if flags:
+            lq_decode_step_ex(self.cfg, self.buf, q, k, v, beta, decay, out, flags, stream)
+        else:
+            lq_decode_step(self.cfg, self.buf, q, k, v, beta, decay, out, stream)
 
     def flush(self, stream=None):
         lq_window_flush(self.cfg, self.buf, stream)

@@ -121,8 +121,10 @@ template <int D, int BITS>
 lq_status launch_decode(const lq_config &c, const DecodeArgs &a, cudaStream_t s) {
     const bool multi = a.tokens > 1;
     const uint32_t smem = decode_smem_bytes(D, a.L, a.F, multi ? a.tokens : 1);
-    auto k = a.map.slots ? (multi ? decode_kernel<D, BITS, true, true> : decode_kernel<D, BITS, true, false>)
-                         : (multi ? decode_kernel<D, BITS, false, true> : decode_kernel<D, BITS, false, false>);
+    auto k = a.map.slots ? (multi ? decode_kernel<D, BITS, true, true, false> : decode_kernel<D, BITS, true, false, false>)
+                         : (multi ? decode_kernel<D, BITS, false, true, false>
+                                  : ((a.flags & kEarlyState) ? decode_kernel<D, BITS, false, false, true>
+                                                             : decode_kernel<D, BITS, false, false, false>));
     cudaError_t e = allow_smem(k, smem);
     if (e != cudaSuccess) return LQ_ERR_CUDA;
     const int threads = D + 64;
@@ -319,10 +321,11 @@ lq_status lq_state_init(const lq_config *cfg, void *state, const float *S0, lq_s
     return dispatch_boundary<1>(c, a, s);
 }
 
-lq_status lq_decode_step(const lq_config *cfg, void *state, const void *q, const void *k,
-                         const void *v, const float *beta, const float *decay, float *out,
-                         lq_stream_t stream) {
+lq_status lq_decode_step_ex(const lq_config *cfg, void *state, const void *q, const void *k,
+                            const void *v, const float *beta, const float *decay, float *out, uint32_t flags,
+                            lq_stream_t stream) {
     lq_status st = check_config(cfg);
+    if (flags & ~kEarlyState) return LQ_ERR_INVALID_ARG;
     if (st != LQ_OK) return st;
     if (!state || !q || !k || !v || !beta || !decay || !out) return LQ_ERR_INVALID_ARG;
     if (!aligned(state, 256) || !aligned(q, 16) || !aligned(k, 16) || !aligned(v, 16) ||
@@ -342,8 +345,14 @@ lq_status lq_decode_step(const lq_config *cfg, void *state, const void *q, const
         return c.dk == 128 ? launch_fp32_decode<128>(c, a, s) : launch_fp32_decode<64>(c, a, s);
     }
     DecodeArgs a{static_cast<uint8_t *>(state), L, make_flags(c), q, k, v, beta, decay, out,
-                 c.num_slots * c.num_heads, SlotMap{nullptr, c.num_heads, c.num_slots}, 1};
+                 c.num_slots * c.num_heads, SlotMap{nullptr, c.num_heads, c.num_slots}, 1, flags};
     return dispatch_decode(c, a, s);
+}
+
+lq_status lq_decode_step(const lq_config *cfg, void *state, const void *q, const void *k,
+                         const void *v, const float *beta, const float *decay, float *out,
+                         lq_stream_t stream) {
+    return lq_decode_step_ex(cfg, state, q, k, v, beta, decay, out, 0u, stream);
 }
 
 lq_status lq_window_flush(const lq_config *cfg, void *state, lq_stream_t stream) {

@@ -129,6 +129,12 @@ __device__ __forceinline__ void mbar_arrive_expect_tx(uint64_t *bar, uint32_t by
                  "r"(bytes) : "memory");
 }
 
+// Expect `bytes` more of transaction on the current phase without arriving.
+__device__ __forceinline__ void mbar_expect_tx(uint64_t *bar, uint32_t bytes) {
+    asm volatile("mbarrier.expect_tx.relaxed.cta.shared::cta.b64 [%0], %1;" ::"r"(smem_u32(bar)), "r"(bytes)
+                 : "memory");
+}
+
 // Test for completion of phase `phase`; the thread may sleep in the barrier
 // for up to ~1 ms (suspend-time hint) while the phase is still open.
 __device__ __forceinline__ bool mbar_try_wait(uint64_t *bar, uint32_t phase) {

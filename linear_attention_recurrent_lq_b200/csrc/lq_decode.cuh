@@ -49,7 +49,14 @@ struct DecodeArgs {
     int num_heads;  // work items: N * H, or active rows * H with a slot map
     SlotMap map;    // heads = H always; slots only in the slot-list instance
     int tokens;     // T consecutive tokens per work item (multi-token instance)
+    uint32_t flags; // kEarlyState (plain rows only)
 };
+
+// Call flag of the plain decode: the kernel enqueued just before this one on
+// the stream does not write the state (it may still be running).  The
+// decode then stages its first blobs and loads their codes before it waits
+// for that kernel; the token's inputs are still read only after the wait.
+constexpr uint32_t kEarlyState = 0x1u;
 
 constexpr int kDotSlots = kMaxWindow + kMaxComp;
 constexpr int kMaxTokens = 8;  // tokens per work item in one multi-token launch
@@ -316,10 +323,13 @@ __device__ __forceinline__ float warp_sum(float x) {
 // SLOTS: work items reach their blobs through A.map.  MULTI: each work item
 // takes A.tokens consecutive tokens (inputs and outputs [rows, T, H, .]),
 // reading its compact state once; token t sees the pairs of tokens < t
-// through the stage, where the epilogue also appends them.  Separate
-// instances, so the plain path carries none of this.
-template <int D, int BITS, bool SLOTS, bool MULTI>
+// through the stage, where the epilogue also appends them.  EARLY (plain
+// rows only, kEarlyState): the first two blobs' state is staged before the
+// wait on the previous kernel.  Separate instances, so the plain path
+// carries none of this.
+template <int D, int BITS, bool SLOTS, bool MULTI, bool EARLY>
 __global__ void __launch_bounds__(D + 64, (SLOTS || MULTI) ? 3 : 0) decode_kernel(DecodeArgs A) {
+    static_assert(!(EARLY && (SLOTS || MULTI)), "early staging is for plain rows");
     constexpr int NC = D;            // consumer threads
     constexpr int LPR = D / 16;      // threads per row, one 16-key chunk each
     constexpr int RPT = D / 16;      // rows per thread (16 row groups)
@@ -374,14 +384,46 @@ __global__ void __launch_bounds__(D + 64, (SLOTS || MULTI) ? 3 : 0) decode_kerne
         fence_mbar_init();
     }
     __syncthreads();
-    // While the previous kernel on the stream drains, start pulling this
-    // CTA's first two blobs (compact state and codes) into L2.  A prefetch
-    // changes no data, so it is safe whatever that kernel writes.  Not
-    // through a slot list: the list would have to be read first, and that
-    // read measured slower than no prefetch at all.
-    if (tid == 0 && !SLOTS)
+    // consumer roles (see below); the codes of the first head are loaded
+    // before the wait in the EARLY instance
+    const int c = tid % LPR, rg = tid / LPR;
+    const uint8_t *code_base = A.state + L.codes_off + c * GB;
+    Group<BITS> cg[RPT];
+    const int b_first = n_mine > 0 ? blob_of(A.map, (int)blockIdx.x) : -1;
+    if (EARLY) {
+        // The previous kernel does not write this state: stage the compact
+        // state and buffered pairs of the first two heads (counts, then bulk
+        // copies on the stages' barriers, without arriving) and load the first
+        // head's codes while that kernel drains.
+        if (warp == COPY_WARP) {
+            if (lane < 2 && lane < n_mine)
+                s_cnt[lane] = *reinterpret_cast<const uint32_t *>(A.state + ((size_t)blockIdx.x + (size_t)lane * G) *
+                                                                                 L.blob + kHdrCount);
+            __syncwarp();
+            if (lane == 0)
+                for (int x = 0; x < 2 && x < n_mine; ++x) {
+                    const uint8_t *blob = A.state + ((size_t)blockIdx.x + (size_t)x * G) * L.blob;
+                    uint8_t *st = stages + (size_t)x * SG.bytes;
+                    const uint32_t cc = s_cnt[x] < (uint32_t)F.window ? s_cnt[x] : 0u;
+                    mbar_expect_tx(&full[x], L.codes_off + cc * L.pair_bytes);
+                    bulk_g2s(st, blob, L.codes_off, &full[x]);
+                    if (cc) bulk_g2s(st + SG.pairs_at, blob + L.pairs_off, cc * L.pair_bytes, &full[x]);
+                }
+            __syncwarp();
+        } else if (warp < COPY_WARP && b_first >= 0) {
+            const uint8_t *cb = code_base + (size_t)b_first * L.blob;
+#pragma unroll
+            for (int m = 0; m < RPT; ++m) load_group<BITS>(cg[m], cb + (size_t)(RPT * rg + m) * L.row_bytes);
+        }
+    } else if (tid == 0 && !SLOTS) {
+        // While the previous kernel on the stream drains, start pulling this
+        // CTA's first two blobs (compact state and codes) into L2.  A prefetch
+        // changes no data, so it is safe whatever that kernel writes.  Not
+        // through a slot list: the list would have to be read first, and that
+        // read measured slower than no prefetch at all.
         for (int it = 0; it < 2 && it < n_mine; ++it)
             bulk_prefetch_l2(A.state + ((size_t)blockIdx.x + (size_t)it * G) * L.blob, L.pairs_off);
+    }
     pdl_wait();
     pdl_trigger();
 
@@ -436,13 +478,17 @@ __global__ void __launch_bounds__(D + 64, (SLOTS || MULTI) ? 3 : 0) decode_kerne
                         continue;
                     }
                     const uint8_t *blob = A.state + (size_t)s_bidx[x] * L.blob;
-                    const uint32_t c = s_cnt[x];
-                    const uint32_t cc = c < (uint32_t)F.window ? c : 0u;
-                    const uint32_t pb = cc * L.pair_bytes;
-                    mbar_arrive_expect_tx(&full[s], L.codes_off + pb +
-                                                        (uint32_t)T * (3 * SG.qkv_bytes + (F.kda ? (uint32_t)D * 4u : 0u)));
-                    bulk_g2s(st, blob, L.codes_off, &full[s]);
-                    if (pb) bulk_g2s(st + SG.pairs_at, blob + L.pairs_off, pb, &full[s]);
+                    const uint32_t in_bytes = (uint32_t)T * (3 * SG.qkv_bytes + (F.kda ? (uint32_t)D * 4u : 0u));
+                    if (EARLY && it < kDecodeStages) {
+                        mbar_arrive_expect_tx(&full[s], in_bytes);  // the state is on its way already
+                    } else {
+                        const uint32_t cnt = s_cnt[x];
+                        const uint32_t cc = cnt < (uint32_t)F.window ? cnt : 0u;
+                        const uint32_t pb = cc * L.pair_bytes;
+                        mbar_arrive_expect_tx(&full[s], L.codes_off + pb + in_bytes);
+                        bulk_g2s(st, blob, L.codes_off, &full[s]);
+                        if (pb) bulk_g2s(st + SG.pairs_at, blob + L.pairs_off, pb, &full[s]);
+                    }
                     for (int t = 0; t < T; ++t) {
                         const size_t r = tok_row(h, t);
                         const size_t qo = r * (size_t)SG.qkv_bytes;
@@ -652,14 +698,9 @@ __global__ void __launch_bounds__(D + 64, (SLOTS || MULTI) ? 3 : 0) decode_kerne
     // ---------------------------------------------------- consumer threads
     // GEMV role: chunk c of rows RPT*rg + m (m < RPT); the per-chunk sums go
     // to shared memory and thread j then owns row j in the epilogue.
-    const int c = tid % LPR, rg = tid / LPR;
     // dot-product role: 8 lanes per job, lane kc takes keys 4*kc + 32*e + (0..3)
     const int kc = tid % 8, jslot = tid / 8;
-    const uint8_t *code_base = A.state + L.codes_off + c * GB;
-
-    Group<BITS> cg[RPT];
-    const int b_first = n_mine > 0 ? blob_of(A.map, (int)blockIdx.x) : -1;
-    if (b_first >= 0) {
+    if (!EARLY && b_first >= 0) {
         const uint8_t *cb = code_base + (size_t)b_first * L.blob;
 #pragma unroll
         for (int m = 0; m < RPT; ++m) load_group<BITS>(cg[m], cb + (size_t)(RPT * rg + m) * L.row_bytes);

@@ -177,3 +177,12 @@ def test_prefill_arguments_rejected_before_launch(B):
 def test_selftest_wait_arguments(B):
     assert B.lib.lq_selftest_wait(None, None) == 1
     assert B.lib.lq_selftest_wait(2, None) == 6
+
+
+def test_decode_step_ex_flags(B):
+    cfg = B.make_config(4, 4)
+    c = ctypes.byref(cfg)
+    ok = (256, 16, 16, 16, 16, 16, 16)
+    assert B.lib.lq_decode_step_ex(c, *ok, 2, None) == 1          # unknown flag bit
+    assert B.lib.lq_decode_step_ex(c, 128, 16, 16, 16, 16, 16, 16, 1, None) == 6
+    assert B.lib.lq_decode_step_ex(c, None, 16, 16, 16, 16, 16, 16, 1, None) == 1

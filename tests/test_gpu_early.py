@@ -1,0 +1,56 @@
+"""The early-state flag of lq_decode_step_ex: with states taking turns on
+the stream (the previous launch never writes the next one's state), a
+window of flagged steps and its flush give, bit for bit, the outputs and
+blobs of unflagged steps."""
+import pytest
+
+from linear_attention_recurrent_lq_b200 import inputs as I
+from tests.gpu_helpers import device_inputs
+
+torch = pytest.importorskip("torch")
+pytestmark = pytest.mark.gpu
+
+NAMES = ("q", "k", "v", "beta", "decay")
+
+
+@pytest.fixture(scope="module", autouse=True)
+def _cuda():
+    if not torch.cuda.is_available():
+        pytest.skip("no CUDA device")
+    from linear_attention_recurrent_lq_b200 import build
+    build.build()
+
+
+@pytest.mark.parametrize("kind,bits", [("gdn_int8_b64h32", 8), ("kda_int8_b128h32", 4),
+                                       ("gdn_int8_b64h32", 6)])
+def test_early_state_steps_equal_plain_steps(kind, bits):
+    from linear_attention_recurrent_lq_b200 import binding as B
+    wl = I.WORKLOADS[kind].replace(batch=7, heads=9, window=8)  # 63 heads: several per CTA
+    L, T = 3, 12  # three layer-states taking turns; a flush after token 8
+    draws = [I.InputStream(wl, stream=l) for l in range(L)]
+    st0 = [s.state() for s in draws]
+    toks = [s.tokens(T) for s in draws]
+    cfg = B.config_for(wl, bits=bits)
+    plain, early = [], []
+    for l in range(L):
+        for group in (plain, early):
+            st = B.LQState(cfg)
+            st.buf.zero_()
+            st.init(torch.from_numpy(st0[l]["S0"]).cuda())
+            group.append(st)
+    dev = [device_inputs(wl, toks[l]) for l in range(L)]
+    outs = {}
+    for name, group, flags in (("plain", plain, 0), ("early", early, B.LQ_STEP_EARLY_STATE)):
+        out = torch.empty((T, L, wl.batch, wl.heads, wl.dv), device="cuda")
+        for t in range(T):
+            for l in range(L):
+                group[l].step(*[dev[l][x][t] for x in NAMES], out[t, l], flags=flags)
+            if t + 1 == wl.window:
+                for l in range(L):
+                    group[l].flush()
+        torch.cuda.synchronize()
+        outs[name] = out
+    assert torch.equal(outs["plain"], outs["early"])
+    for a, b in zip(plain, early):
+        assert torch.equal(a.buf, b.buf)
+        assert b.check() == 0
