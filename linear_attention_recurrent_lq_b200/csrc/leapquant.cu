@@ -548,7 +548,7 @@ const char *lq_status_string(lq_status s) {
     switch (s) {
         case LQ_OK: return "ok";
         case LQ_ERR_INVALID_ARG: return "invalid argument";
-        case LQ_ERR_UNSUPPORTED: return "configuration not supported by this build";
+        case LQ_ERR_UNSUPPORTED: return "configuration not supported by this library";
         case LQ_ERR_CUDA: return "CUDA error";
         case LQ_ERR_WINDOW_FULL: return "decode step into a full window (flush every W steps)";
         case LQ_ERR_RANGE: return "a gate (decay) was negative or NaN";
