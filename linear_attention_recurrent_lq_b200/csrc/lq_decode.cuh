@@ -15,11 +15,14 @@
 //     u_t = beta (v - a),   o_t = b + (k . q) u_t,
 // and the pair (khat_t = k / g_t, u_t) is appended.
 //
-// Persistent kernel, one CTA = D consumer threads + one producer warp, each
-// CTA walking a strided list of (slot, head) blobs:
-//  * the producer warp bulk-copies each blob's small, variable-size parts
+// Persistent kernel, one CTA = D consumer threads + a copy warp + a prep
+// warp, each CTA walking a strided list of (slot, head) blobs:
+//  * the copy warp bulk-copies each blob's small, variable-size parts
 //    (header, decay product, scales, compensators, the buffered pairs) and the
 //    token's q, k, v into a two-stage shared-memory ring (mbarrier-tracked);
+//  * the prep warp, one head ahead, checks the header and forms the decayed
+//    and quantized vectors of the head (and moves the window frame when a
+//    decay product leaves its range);
 //  * the codes (the bulk of the state) go straight from global memory into
 //    registers: a consumer thread holds its D/16 16-code groups of the current
 //    blob and, as it consumes group m, issues the load of group m of the next
