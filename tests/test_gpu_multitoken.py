@@ -24,6 +24,7 @@ CASES = {
     "kda_int4": (W["kda_int8_b128h32"].replace(batch=5, heads=3), 4),
     "gdn_int6_d64": (W["gdn_int8_b64h32"].replace(batch=5, heads=3, dk=64, dv=64), 6),
     "kda_int8_f16": (W["kda_int8_b128h32"].replace(batch=5, heads=3, scale_dtype="f16"), 8),
+    "gdn_int8_d64_f32in": (W["gdn_int8_b64h32"].replace(batch=5, heads=3, dk=64, dv=64, in_dtype="f32"), 8),
 }
 NAMES = ("q", "k", "v", "beta", "decay")
 

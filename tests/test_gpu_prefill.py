@@ -169,3 +169,27 @@ def test_full_size_prefill_sampled_heads():
         r = compare_compressed(p, S_gpu[x], blob.parse(p, blobs[h]))
         assert r["flips"] == 0, (h, r)
     assert st.check() == 0
+
+
+def test_one_token_prompts_and_empty_prompts():
+    """T = 1, and a length list of zeros (every row keeps S0: the blob equals
+    the init's, the outputs are zero)."""
+    wl, bits = CASES["gdn_int8"]
+    d = I.draw(wl, 1)
+    S0 = torch.from_numpy(d["S0"]).cuda()
+    st = _state(wl, bits)
+    out = torch.empty((wl.batch, 1, wl.heads, wl.dv), dtype=torch.float32, device="cuda")
+    st.prefill(1, *_row_major(wl, d, 1), S0=S0, out=out)
+    torch.cuda.synchronize()
+    nh, H = wl.batch * wl.heads, wl.heads
+    o_ref, _, _ = oracle.prefill(_params(wl, bits), *oracle_inputs(wl, d, np.arange(nh), 1))
+    assert rel_l2(out.transpose(0, 1).cpu().numpy().reshape(1, nh, wl.dv), o_ref) < REL_L2
+    z, ini = _state(wl, bits), _state(wl, bits)
+    outz = torch.full((wl.batch, 1, wl.heads, wl.dv), float("nan"), device="cuda")
+    z.prefill(1, *_row_major(wl, d, 1), S0=S0, out=outz,
+              lengths=torch.zeros(wl.batch, dtype=torch.int32, device="cuda"))
+    ini.init(S0)
+    torch.cuda.synchronize()
+    assert not outz.any() and not outz.isnan().any()
+    assert torch.equal(z.buf, ini.buf)
+    assert z.check() == 0 and st.check() == 0

@@ -22,6 +22,7 @@ CASES = {
     "gdn_int8": (W["gdn_int8_b64h32"].replace(batch=6, heads=3), 8),
     "kda_int4": (W["kda_int8_b128h32"].replace(batch=6, heads=3), 4),
     "gdn_int6_d64": (W["gdn_int8_b64h32"].replace(batch=6, heads=3, dk=64, dv=64), 6),
+    "kda_int8_f16": (W["kda_int8_b128h32"].replace(batch=6, heads=3, scale_dtype="f16"), 8),
 }
 
 
