@@ -14,7 +14,17 @@ the L window flushes.  Rotating L = 8 layers keeps the working set (~0.6 GB of
 state) well above the 126 MB L2, so every token re-reads its state from HBM;
 no L2 flush is needed.  Inputs are seeded synthetic draws, resident in HBM
 before timing; every step reuses the same window of inputs on an evolving
-state.
+state.  The decodes go through lq_decode_step_ex with LQ_STEP_EARLY_STATE
+when two or more layer-states rotate (the launch before each decode is then
+always another state's).
+
+Besides the headline line, the JSON carries, each timed on its own:
+fp32_state (the FP32-state kernel on the same inputs), per_step_baselines
+(BF16, FP8 E4M3 and INT8 states stored every token), multi_token (T tokens
+per launch), prefill (a 256-token prompt then compression), serving_slots
+(decode and flush through a shuffled slot list), e2e (host buffers, the
+transfers overlapped with the kernels) and cpu_baseline (the oracle on the
+host cores).
 
 Launch: python bench.py [--gpus N --steps K --warmup W]; for N > 1 under
 torch.distributed.run, one process per GPU, each rank advancing its own
