@@ -129,6 +129,20 @@ def per_step_bytes(wl, fmt):
     return 2 * state + f["inputs"] + f["out"]
 
 
+def state_memory(wl, B):
+    """Bytes of state per (sequence, head): the LeapQuant blob (window buffer
+    included), its compact part alone (what a flushed prefix-cache entry
+    holds), and the FP32-state blob; plus the whole layer at this workload."""
+    lq = B.lq_state_bytes(B.config_for(wl))
+    f32 = B.lq_state_bytes(B.config_for(wl, bits=32))
+    f = field_bytes(wl)
+    compact = f["hdr"] + f["meta"] + f["qs"] + f["sm"] + f["cvec"] + f["codes"] + f["g"]
+    nh = wl.batch * wl.heads
+    return {"leapquant_blob_bytes": lq, "leapquant_compact_bytes": compact, "fp32_blob_bytes": f32,
+            "layer_leapquant_mb": nh * lq / 1e6, "layer_fp32_mb": nh * f32 / 1e6,
+            "compact_vs_fp32": f32 / compact}
+
+
 def fp32_bytes(wl):
     """FP32-state step per head: read and write the dense state, read inputs,
     write the output."""
@@ -574,6 +588,7 @@ def main_ours(args):
                      "flush_avg_launch_us": fl_ms * 1e3,
                      "flush_algorithmic_bytes_per_launch": nh * flush_bytes(wl)},
         "gpu_launches": args.steps * arm.launches_per_step(),
+        "state_memory": state_memory(wl, B),
         "clocks": clk,
     }
 

@@ -65,3 +65,15 @@ def test_source_hash_ignores_comments(bench):
     assert bench.strip_comments(a) == bench.strip_comments(b)
     assert bench.strip_comments(a) != bench.strip_comments(c)
     assert len(bench.kernel_source_sha()) == 16
+
+
+def test_state_memory_figures(bench, wl):
+    from linear_attention_recurrent_lq_b200 import build
+    build.build()
+    from linear_attention_recurrent_lq_b200 import binding as B
+    m = bench.state_memory(wl, B)
+    assert m["leapquant_blob_bytes"] == 36096
+    assert m["leapquant_compact_bytes"] == 20 + 16 + 512 + 512 + 2048 + 16384
+    assert m["fp32_blob_bytes"] >= 4 * 128 * 128
+    assert 3.0 < m["compact_vs_fp32"] < 3.5
+    assert m["layer_leapquant_mb"] == 2048 * 36096 / 1e6
