@@ -61,6 +61,9 @@ MUTATIONS = {
     "prefill reads the decay of the wrong token": (
         "ad[i] = kda ? decay[th * dk + i] : decay[th];",
         "ad[i] = kda ? decay[(th % nh) * dk + i] : decay[th % nh];"),
+    "prefill starts from a zero state": (
+        "for (int x = 0; x < dk * dv; ++x) S[x] = (double)S0[(size_t)h * dk * dv + x];\n        for (int t = 0; t < T; ++t) {\n            size_t th = (size_t)t * nh + h;\n            if (t >= n) {",
+        "for (int x = 0; x < dk * dv; ++x) S[x] = 0.0;\n        for (int t = 0; t < T; ++t) {\n            size_t th = (size_t)t * nh + h;\n            if (t >= n) {"),
     "per-step state not stored after the token": (
         "                per_step_store(p, S, buf32, qs, val);\n            } else",
         "                ;\n            } else"),
