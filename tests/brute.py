@@ -98,3 +98,56 @@ def run(S0, q, k, v, beta, a, W, bits, r, smoothing, scale_f16=False):
         if quant and (t + 1) % W == 0:
             S = requant(S)
     return np.array(outs), S
+
+
+def f32_round(x):
+    """Round an exact rational (fractions.Fraction or int) to the nearest
+    binary32, ties to even, with gradual underflow; written from the format's
+    definition (24 significant bits, smallest normal 2^-126) with integer
+    arithmetic only, so no intermediate rounding can creep in."""
+    from fractions import Fraction
+    x = Fraction(x)
+    if x == 0:
+        return np.float32(0.0)
+    sign = -1 if x < 0 else 1
+    a = abs(x)
+    # e = floor(log2(a))
+    e = a.numerator.bit_length() - a.denominator.bit_length()
+    if Fraction(2) ** e > a:
+        e -= 1
+    e = max(e, -126)
+    quantum = Fraction(2) ** (e - 23)
+    n, rem = divmod(a, quantum)        # a = n * quantum + rem, 0 <= rem < quantum
+    n = int(n)
+    if rem * 2 > quantum or (rem * 2 == quantum and n % 2 == 1):
+        n += 1
+    return np.float32(sign * float(n * quantum))
+
+
+def reconstruct_f32(codes, qs, sm, meta, vec, pairs, g):
+    """The FP32 window-end state, written independently of the C oracle:
+    S_ij = g_i * ( ((qs_j * C_ji) * sm_i) + compensators in round order
+                   + fused multiply-add over the pairs in buffer order ),
+    each operation one FP32 rounding.  The fused multiply-add is taken
+    exactly in rationals, then rounded once (f32_round).
+    codes [dv, dk] (value-major); meta / vec as the compressor returns them;
+    pairs [count, dk + dv] (khat then u); g [dk]."""
+    from fractions import Fraction
+    dv, dk = codes.shape
+    S = np.zeros((dk, dv), np.float32)
+    for i in range(dk):
+        for j in range(dv):
+            acc = (np.float32(qs[j]) * np.float32(codes[j, i])) * np.float32(sm[i])
+            for c, m in enumerate(meta):
+                m = int(m)
+                if m == NONE:
+                    continue
+                if m & KIND_COL:
+                    if (m & 0x7FFFFFFF) == j:
+                        acc = np.float32(acc + np.float32(vec[c][i]))
+                elif m == i:
+                    acc = np.float32(acc + np.float32(vec[c][j]))
+            for pr in pairs:
+                acc = f32_round(Fraction(float(pr[i])) * Fraction(float(pr[dk + j])) + Fraction(float(acc)))
+            S[i, j] = np.float32(g[i]) * acc
+    return S

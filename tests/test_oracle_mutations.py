@@ -67,6 +67,27 @@ MUTATIONS = {
     "per-step state not stored after the token": (
         "                per_step_store(p, S, buf32, qs, val);\n            } else",
         "                ;\n            } else"),
+    "rebuild drops the decay": ("S[i * dv + j] = g[i] * acc;", "S[i * dv + j] = acc;"),
+    "rebuild applies the decay per value column": ("S[i * dv + j] = g[i] * acc;",
+                                                   "S[i * dv + j] = g[j] * acc;"),
+    "rebuild adds a column compensator along a row": (
+        "if ((int)(meta[c] & 0x7FFFFFFFu) == j) acc = acc + w[i];",
+        "if ((int)(meta[c] & 0x7FFFFFFFu) == i) acc = acc + w[j];"),
+    "rebuild drops the compensators": ("if ((int)meta[c] == i) acc = acc + w[j];",
+                                       "if ((int)meta[c] == i) acc = acc + 0.0f;"),
+    "rebuild takes the pairs in reverse order": (
+        "acc = fmaf(pairs[(size_t)m * pd + i], pairs[(size_t)m * pd + dk + j], acc);",
+        "acc = fmaf(pairs[(size_t)(count - 1 - m) * pd + i], pairs[(size_t)(count - 1 - m) * pd + dk + j], acc);"),
+    "rebuild multiplies then adds the pair terms": (
+        "acc = fmaf(pairs[(size_t)m * pd + i], pairs[(size_t)m * pd + dk + j], acc);",
+        "acc = acc + pairs[(size_t)m * pd + i] * pairs[(size_t)m * pd + dk + j];"),
+    "rebuild reads u at the wrong pair offset": (
+        "pairs[(size_t)m * pd + dk + j], acc);", "pairs[(size_t)m * pd + dv + j], acc);"),
+    "rebuild drops the last pair": ("for (int m = 0; m < count; ++m)\n                acc = fmaf(",
+                                    "for (int m = 0; m + 1 < count; ++m)\n                acc = fmaf("),
+    "rebuild adds the compensators in reverse round order": (
+        "for (int c = 0; c < p->num_comp; ++c) {\n                if (meta[c] == LQO_NONE) continue;\n                const float *w = vec + (size_t)c * maxd;\n                if (meta[c] & LQO_KIND_COL) {\n                    if ((int)(meta[c] & 0x7FFFFFFFu) == j)",
+        "for (int c = p->num_comp - 1; c >= 0; --c) {\n                if (meta[c] == LQO_NONE) continue;\n                const float *w = vec + (size_t)c * maxd;\n                if (meta[c] & LQO_KIND_COL) {\n                    if ((int)(meta[c] & 0x7FFFFFFFu) == j)"),
 }
 
 PIN_TESTS = [getattr(pins, n) for n in dir(pins) if n.startswith("test_")]

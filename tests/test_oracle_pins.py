@@ -595,3 +595,88 @@ def test_prefill_one_token_from_zero_writes_beta_k_v(oracle_lib):
                              np.array([[0.5]], np.float32), np.array([[0.75]], np.float32))
     np.testing.assert_array_equal(S[0], 0.5 * np.outer(k[0, 0], v[0, 0]))
     np.testing.assert_array_equal(o[0, 0], 0.5 * float(k[0, 0] @ q[0, 0]) * v[0, 0])
+
+
+# --------------------------------------------------------------------------
+# the FP32 window-end rebuild (what the flush requantizes and dequant returns)
+
+def _hexf(x):
+    return np.array([[float.fromhex(v) for v in row] for row in x] if isinstance(x[0], list)
+                    else [float.fromhex(v) for v in x], np.float32)
+
+
+def test_golden_rebuild_order(oracle_lib):
+    """Hand-derived 3 x 2 rebuild whose FP32 result depends on the order the
+    rule fixes: fused pair terms, compensators in round order, pairs in buffer
+    order, the decay of the key row applied last (tests/golden)."""
+    g = json.load(open(os.path.join(GOLDEN, "rebuild_3x2_f32.json")))
+    pr = g["params"]
+    p = oracle.Params(dk=pr["dk"], dv=pr["dv"], bits=pr["bits"], num_comp=pr["num_comp"])
+    codes = np.array(g["codes_value_major"], np.int8)
+    args = (codes, _hexf(g["qs"]), _hexf(g["sm"]), np.array(g["meta"], np.uint32), _hexf(g["vec"]),
+            _hexf(g["pairs_khat_then_u"]), _hexf(g["g"]))
+    expect = _hexf(g["S"])
+    np.testing.assert_array_equal(oracle.reconstruct_f32(p, *args), expect)
+    np.testing.assert_array_equal(brute.reconstruct_f32(*args), expect)
+
+
+def _rand_compact(rng, dk, dv, r, count, bits=8):
+    """A compressed random head plus `count` random pairs and a decay vector."""
+    S = _rand_state(rng, dk, dv, rows=(1,), cols=(dv - 2,), gain=30.0).astype(np.float32)
+    p = oracle.Params(dk=dk, dv=dv, bits=bits, num_comp=r, window=max(count, 1))
+    c = oracle.compress(p, S)
+    pairs = np.concatenate([rng.normal(size=(count, dk)), rng.normal(0, 0.3, (count, dv))],
+                           axis=1).astype(np.float32)
+    g = rng.uniform(0.2, 1.0, dk).astype(np.float32)
+    return p, c, pairs, g
+
+
+def test_rebuild_within_fp32_rounding_bound_of_exact_sum(oracle_lib):
+    """Against the exact (FP64) matrix the blob stands for,
+    diag(g) (Dequant(compact) + sum_m khat_m u_m^T): each entry is within the
+    forward error bound of the FP32 evaluation.  The rebuild rounds once for
+    qs*C (the power-of-two smoothing scale multiplies exactly), once per
+    compensator addition and fused pair term, and once for the decay:
+        |S32 - S| <= (n + 2) 2^-24 |g_i| (|B_ij| + sum of |added terms|),
+    with n the number of additions.  A dropped, doubled or misplaced term
+    moves an entry by far more."""
+    rng = np.random.default_rng(90)
+    u = 2.0 ** -24
+    for dk, dv, r, count in ((16, 16, 3, 5), (24, 16, 4, 9), (8, 8, 0, 0), (32, 32, 2, 15)):
+        p, c, pairs, g = _rand_compact(rng, dk, dv, r, count)
+        S32 = oracle.reconstruct_f32(p, c["codes"], c["qs"], c["sm"], c["meta"], c["vec"], pairs, g)
+        base = (c["sm"].astype(np.float64)[:, None] * c["qs"].astype(np.float64)[None, :]
+                * c["codes"].T.astype(np.float64))
+        mag = np.abs(base)
+        inner = oracle.dequant(p, c["codes"], c["qs"], c["sm"], c["meta"], c["vec"])
+        mag = mag + np.abs(inner - base)        # the compensator entries (exact in FP64)
+        for m in range(count):
+            t = np.outer(pairs[m, :dk].astype(np.float64), pairs[m, dk:].astype(np.float64))
+            inner = inner + t
+            mag = mag + np.abs(t)
+        exact = g.astype(np.float64)[:, None] * inner
+        n = 1 + r + count
+        bound = 1.0001 * (n + 2) * u * g.astype(np.float64)[:, None] * mag + 1e-45
+        err = np.abs(S32.astype(np.float64) - exact)
+        assert np.all(err <= bound), (dk, dv, r, count, float(np.max(err / bound)))
+        if count:   # the bound is far tighter than one pair's contribution
+            one = np.abs(g.astype(np.float64)[:, None] * np.outer(pairs[-1, :dk], pairs[-1, dk:]))
+            assert np.median(one / bound) > 100
+
+
+def test_rebuild_matches_brute_force_bit_for_bit(oracle_lib):
+    """Random tiny heads, non-square, f32 scales: the C rebuild equals an
+    independent NumPy restatement (exact rational fused multiply-add, one
+    rounding per operation) in every bit."""
+    rng = np.random.default_rng(91)
+    for trial in range(12):
+        dk, dv = (int(x) for x in rng.choice([4, 6, 8], 2))
+        if dv > dk:
+            dk, dv = dv, dk
+        r = int(rng.integers(0, 4))
+        count = int(rng.integers(0, 6))
+        p, c, pairs, g = _rand_compact(rng, dk, dv, r, count, bits=int(rng.choice([8, 6, 4])))
+        args = (c["codes"], c["qs"], c["sm"], c["meta"], c["vec"], pairs, g)
+        a = oracle.reconstruct_f32(p, *args)
+        b = brute.reconstruct_f32(*args)
+        np.testing.assert_array_equal(a.view(np.uint32), b.view(np.uint32))
