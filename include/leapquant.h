@@ -136,11 +136,15 @@ typedef struct lq_config {
                             scale_dtype are then not used)                    */
 } lq_config;
 
-/* LQ_OK if the configuration is valid and built, else why not.  Host only. */
+/* LQ_OK if the configuration is valid and built, else why not.  Host only.
+ * Library infrastructure: no passage of the pages defines it. */
 LQ_API lq_status lq_validate_config(const lq_config *cfg);
 
 /* Bytes of one (slot, head) blob, a multiple of 256; 0 for an invalid or
- * unsupported configuration.  Host only. */
+ * unsupported configuration.  Host only.  The blob holds what the news post's
+ * per-window, Compensator Tokens and residual smoothing paragraphs keep per
+ * head (low-bit codes, scales, FP32 compensator lines, the window's FP32
+ * pairs); its size is this library's layout, which no passage fixes. */
 LQ_API size_t lq_state_bytes(const lq_config *cfg);
 
 /* Enter a sequence: compress N*H dense FP32 states into the blobs.
@@ -187,24 +191,35 @@ LQ_API lq_status lq_window_flush(const lq_config *cfg, void *state, lq_stream_t 
 /* Write the dense FP32 state each blob stands for, pending pairs included:
  *   S_out [N, H, dk, dv] f32, out.
  * Evaluated exactly as the flush rebuilds it before requantizing, so the
- * flush of a blob compresses bit-for-bit this matrix. */
+ * flush of a blob compresses bit-for-bit this matrix.  Source: the state is
+ * the fixed low-bit part plus the cached high-precision updates (news post,
+ * per-window paragraph) plus the compensator pairs (Compensator Tokens
+ * paragraph); the FP32 evaluation order is this library's reading:
+ *   S_ij = g_i * ( ((qs_j C_ji) sm_i) + compensators in round order
+ *                  + fused multiply-add over the pairs in buffer order ). */
 LQ_API lq_status lq_dequant_state(const lq_config *cfg, const void *state, float *S_out,
                            lq_stream_t stream);
 
 /* Synchronize `stream`, OR the status words of all N*H blobs and map them to
  * the first set error (WINDOW_FULL, RANGE, TIMEOUT, CORRUPT).  `state` is a
- * device pointer; the read uses one strided device-to-host copy. */
+ * device pointer; the read uses one strided device-to-host copy.  Library
+ * infrastructure (failure detection): no passage of the pages defines it. */
 LQ_API lq_status lq_check_status(const lq_config *cfg, const void *state, lq_stream_t stream);
 
 /* lq_decode_step with call flags:
- *   LQ_STEP_EARLY_STATE  the kernel enqueued on `stream` just before this
- *      call does not write `state` (it may still be running when this one
- *      starts: the library launches with programmatic dependent launch).
- *      The step then stages its first blobs' compact state and codes while
- *      that kernel drains; q, k, v, beta and decay are still read only after
- *      it has completed.  True in a model when the previous kernel is, say,
- *      the projection that produces q, k, v; false when two steps on the same
- *      state follow each other directly.  A wrong promise reads stale state.
+ *   LQ_STEP_EARLY_STATE  no kernel that may still be running when this step
+ *      starts writes `state`.  The library launches with programmatic
+ *      dependent launch, so the step can start while the kernel enqueued just
+ *      before it drains; it then stages its first blobs' compact state and
+ *      codes at once, and reads q, k, v, beta and decay only after that
+ *      kernel has completed.  The promise holds when (a) the kernel just
+ *      before this call does not write `state`, and (b) that kernel is not a
+ *      programmatic-dependent launch, or triggers its dependents only after
+ *      its own dependency wait (every kernel of this library does), so that
+ *      no kernel further back can still be running.  True in a model when
+ *      the previous kernel is, say, the projection that produces q, k, v;
+ *      false when two steps on the same state follow each other directly.  A
+ *      wrong promise reads stale state.
  * Other bits: LQ_ERR_INVALID_ARG.  The flag changes nothing for bits = 32
  * and per_step states. */
 #define LQ_STEP_EARLY_STATE 0x1u
@@ -326,7 +341,7 @@ LQ_API lq_status lq_copy_slots(const lq_config *cfg, void *dst, int dst_num_slot
  * Enqueued on `stream`; the call does not wait. */
 LQ_API lq_status lq_selftest_wait(uint32_t *status, lq_stream_t stream);
 
-/* Static text for a status code. */
+/* Static text for a status code.  Library infrastructure. */
 LQ_API const char *lq_status_string(lq_status s);
 
 #ifdef __cplusplus

@@ -120,6 +120,70 @@ def _ptr(x) -> int | None:
     return x.data_ptr()
 
 
+# ---- tensor checks -------------------------------------------------------
+# The C library trusts the shapes it is given: an undersized or mistyped
+# buffer, or one on another device, would make a kernel read or write out of
+# bounds.  Every torch tensor is therefore checked here, before the call, for
+# its element type, its element count against cfg and its device (the GPU
+# that is current, where the library launches).  Raw integer addresses are
+# passed through unchecked: their owner vouches for them.
+
+def _dt(name):
+    import torch
+    return {"f32": torch.float32, "bf16": torch.bfloat16, "i32": torch.int32, "u8": torch.uint8}[name]
+
+
+def _in_dt(cfg) -> str:
+    return "bf16" if cfg.in_dtype else "f32"
+
+
+def _validate(*specs):
+    """Check (tensor, what, dtype(s), numel, at_least) specs: first every
+    element type and count, then that every tensor sits on the current CUDA
+    device.  ValueError on the first mismatch; None and integer addresses
+    pass."""
+    import torch
+    ts = [sp for sp in specs if sp[0] is not None and not isinstance(sp[0], int)]
+    for x, what, dtype, numel, at_least in ts:
+        want = dtype if isinstance(dtype, tuple) else (dtype,)
+        if x.dtype not in tuple(_dt(d) for d in want):
+            raise ValueError(f"{what}: dtype {x.dtype}, expected {' or '.join(want)}")
+        if numel is not None:
+            n = x.numel()
+            if (n < numel) if at_least else (n != numel):
+                raise ValueError(f"{what}: {n} elements, expected {'at least ' if at_least else ''}{numel}")
+    for x, what, *_ in ts:
+        if x.device.type != "cuda":
+            raise ValueError(f"{what}: on {x.device}, expected a CUDA tensor")
+        dev = torch.cuda.current_device()
+        if x.device.index != dev:
+            raise ValueError(f"{what}: on cuda:{x.device.index}, but the library launches on cuda:{dev}")
+
+
+def _spec(x, what, dtype, numel=None, at_least=False):
+    return (x, what, dtype, numel, at_least)
+
+
+def _state_spec(cfg, state, num_slots=None, what="state"):
+    n = cfg.num_slots if num_slots is None else num_slots
+    bb = lib.lq_state_bytes(ctypes.byref(cfg))
+    return _spec(state, what, "u8", n * cfg.num_heads * bb if bb else None, at_least=True)
+
+
+def _rows_specs(cfg, rows: int, T: int, q, k, v, beta, decay, out):
+    H, dk, dv = cfg.num_heads, cfg.dk, cfg.dv
+    n = rows * T * H
+    return [_spec(q, "q", _in_dt(cfg), n * dk), _spec(k, "k", _in_dt(cfg), n * dk),
+            _spec(v, "v", _in_dt(cfg), n * dv), _spec(beta, "beta", "f32", n),
+            _spec(decay, "decay", "f32", n * (dk if cfg.decay_kind == 1 else 1)),
+            _spec(out, "out", "f32", n * dv)]
+
+
+def _dense_spec(cfg, x, what, rows):
+    return _spec(x, what, "f32", rows * cfg.num_heads * cfg.dk * cfg.dv)
+
+
+
 def _stream(stream) -> int | None:
     if stream is None:
         import torch
@@ -152,11 +216,13 @@ def lq_state_bytes(cfg: lq_config) -> int:
 
 
 def lq_state_init(cfg, state, S0, stream=None):
+    _validate(_state_spec(cfg, state), _dense_spec(cfg, S0, "S0", cfg.num_slots))
     _check(lib.lq_state_init(ctypes.byref(cfg), _ptr(state), _ptr(S0), _stream(stream)),
            "lq_state_init")
 
 
 def lq_decode_step(cfg, state, q, k, v, beta, decay, out, stream=None):
+    _validate(_state_spec(cfg, state), *_rows_specs(cfg, cfg.num_slots, 1, q, k, v, beta, decay, out))
     _check(lib.lq_decode_step(ctypes.byref(cfg), _ptr(state), _ptr(q), _ptr(k), _ptr(v),
                               _ptr(beta), _ptr(decay), _ptr(out), _stream(stream)),
            "lq_decode_step")
@@ -166,22 +232,26 @@ LQ_STEP_EARLY_STATE = 0x1
 
 
 def lq_decode_step_ex(cfg, state, q, k, v, beta, decay, out, flags=0, stream=None):
+    _validate(_state_spec(cfg, state), *_rows_specs(cfg, cfg.num_slots, 1, q, k, v, beta, decay, out))
     _check(lib.lq_decode_step_ex(ctypes.byref(cfg), _ptr(state), _ptr(q), _ptr(k), _ptr(v),
                                  _ptr(beta), _ptr(decay), _ptr(out), int(flags), _stream(stream)),
            "lq_decode_step_ex")
 
 
 def lq_window_flush(cfg, state, stream=None):
+    _validate(_state_spec(cfg, state))
     _check(lib.lq_window_flush(ctypes.byref(cfg), _ptr(state), _stream(stream)), "lq_window_flush")
 
 
 def lq_dequant_state(cfg, state, S_out, stream=None):
+    _validate(_state_spec(cfg, state), _dense_spec(cfg, S_out, "S_out", cfg.num_slots))
     _check(lib.lq_dequant_state(ctypes.byref(cfg), _ptr(state), _ptr(S_out), _stream(stream)),
            "lq_dequant_state")
 
 
 def lq_check_status(cfg, state, stream=None) -> int:
     """Synchronizes the stream; returns the status code (does not raise)."""
+    _validate(_state_spec(cfg, state))
     return lib.lq_check_status(ctypes.byref(cfg), _ptr(state), _stream(stream))
 
 
@@ -189,23 +259,37 @@ def _n(slots) -> int:
     return 0 if slots is None else int(slots.numel()) if hasattr(slots, "numel") else len(slots)
 
 
+def _prefill_specs(cfg, rows, tokens, q, k, v, beta, decay, S0, lengths, out, S_final):
+    T = max(int(tokens), 0)
+    return _rows_specs(cfg, rows, T, q, k, v, beta, decay, out) + [
+        _dense_spec(cfg, S0, "S0", rows), _dense_spec(cfg, S_final, "S_final", rows),
+        _spec(lengths, "lengths", "i32", rows)]
+
+
 def lq_state_init_slots(cfg, state, slots, S0, stream=None):
+    _validate(_state_spec(cfg, state), _spec(slots, "slots", "i32"), _dense_spec(cfg, S0, "S0", _n(slots)))
     _check(lib.lq_state_init_slots(ctypes.byref(cfg), _ptr(state), _ptr(slots), _n(slots), _ptr(S0),
                                    _stream(stream)), "lq_state_init_slots")
 
 
 def lq_decode_step_slots(cfg, state, slots, q, k, v, beta, decay, out, stream=None):
+    _validate(_state_spec(cfg, state), _spec(slots, "slots", "i32"),
+              *_rows_specs(cfg, _n(slots), 1, q, k, v, beta, decay, out))
     _check(lib.lq_decode_step_slots(ctypes.byref(cfg), _ptr(state), _ptr(slots), _n(slots), _ptr(q),
                                     _ptr(k), _ptr(v), _ptr(beta), _ptr(decay), _ptr(out),
                                     _stream(stream)), "lq_decode_step_slots")
 
 
 def lq_decode_steps(cfg, state, tokens, q, k, v, beta, decay, out, stream=None):
+    _validate(_state_spec(cfg, state),
+              *_rows_specs(cfg, cfg.num_slots, max(int(tokens), 0), q, k, v, beta, decay, out))
     _check(lib.lq_decode_steps(ctypes.byref(cfg), _ptr(state), int(tokens), _ptr(q), _ptr(k), _ptr(v),
                                _ptr(beta), _ptr(decay), _ptr(out), _stream(stream)), "lq_decode_steps")
 
 
 def lq_decode_steps_slots(cfg, state, slots, tokens, q, k, v, beta, decay, out, stream=None):
+    _validate(_state_spec(cfg, state), _spec(slots, "slots", "i32"),
+              *_rows_specs(cfg, _n(slots), max(int(tokens), 0), q, k, v, beta, decay, out))
     _check(lib.lq_decode_steps_slots(ctypes.byref(cfg), _ptr(state), _ptr(slots), _n(slots), int(tokens),
                                      _ptr(q), _ptr(k), _ptr(v), _ptr(beta), _ptr(decay), _ptr(out),
                                      _stream(stream)), "lq_decode_steps_slots")
@@ -213,6 +297,8 @@ def lq_decode_steps_slots(cfg, state, slots, tokens, q, k, v, beta, decay, out, 
 
 def lq_prefill(cfg, state, tokens, q, k, v, beta, decay, S0=None, lengths=None, out=None, S_final=None,
                stream=None):
+    _validate(_state_spec(cfg, state),
+              *_prefill_specs(cfg, cfg.num_slots, tokens, q, k, v, beta, decay, S0, lengths, out, S_final))
     _check(lib.lq_prefill(ctypes.byref(cfg), _ptr(state), int(tokens), _ptr(lengths), _ptr(S0), _ptr(q),
                           _ptr(k), _ptr(v), _ptr(beta), _ptr(decay), _ptr(out), _ptr(S_final),
                           _stream(stream)), "lq_prefill")
@@ -220,6 +306,8 @@ def lq_prefill(cfg, state, tokens, q, k, v, beta, decay, S0=None, lengths=None, 
 
 def lq_prefill_slots(cfg, state, slots, tokens, q, k, v, beta, decay, S0=None, lengths=None, out=None,
                      S_final=None, stream=None):
+    _validate(_state_spec(cfg, state), _spec(slots, "slots", "i32"),
+              *_prefill_specs(cfg, _n(slots), tokens, q, k, v, beta, decay, S0, lengths, out, S_final))
     _check(lib.lq_prefill_slots(ctypes.byref(cfg), _ptr(state), _ptr(slots), _n(slots), int(tokens),
                                 _ptr(lengths), _ptr(S0), _ptr(q), _ptr(k), _ptr(v), _ptr(beta),
                                 _ptr(decay), _ptr(out), _ptr(S_final), _stream(stream)),
@@ -227,6 +315,7 @@ def lq_prefill_slots(cfg, state, slots, tokens, q, k, v, beta, decay, S0=None, l
 
 
 def lq_window_flush_slots(cfg, state, slots, stream=None):
+    _validate(_state_spec(cfg, state), _spec(slots, "slots", "i32"))
     _check(lib.lq_window_flush_slots(ctypes.byref(cfg), _ptr(state), _ptr(slots), _n(slots),
                                      _stream(stream)), "lq_window_flush_slots")
 
@@ -234,6 +323,8 @@ def lq_window_flush_slots(cfg, state, slots, stream=None):
 def lq_copy_slots(cfg, dst, dst_num_slots, dst_slots, src, src_num_slots, src_slots, stream=None):
     if _n(dst_slots) != _n(src_slots):
         raise ValueError("dst_slots and src_slots must have the same length")
+    _validate(_state_spec(cfg, dst, int(dst_num_slots), "dst"), _state_spec(cfg, src, int(src_num_slots), "src"),
+              _spec(dst_slots, "dst_slots", "i32"), _spec(src_slots, "src_slots", "i32"))
     _check(lib.lq_copy_slots(ctypes.byref(cfg), _ptr(dst), int(dst_num_slots), _ptr(dst_slots),
                              _ptr(src), int(src_num_slots), _ptr(src_slots), _n(src_slots),
                              _stream(stream)), "lq_copy_slots")
@@ -241,6 +332,7 @@ def lq_copy_slots(cfg, dst, dst_num_slots, dst_slots, src, src_num_slots, src_sl
 
 def lq_selftest_wait(status, stream=None):
     """Device diagnostic: a bounded wait that runs out writes LQ_DEV_TIMEOUT to status."""
+    _validate(_spec(status, "status", "i32", 1, at_least=True))
     _check(lib.lq_selftest_wait(_ptr(status), _stream(stream)), "lq_selftest_wait")
 
 

@@ -186,3 +186,66 @@ def test_decode_step_ex_flags(B):
     assert B.lib.lq_decode_step_ex(c, *ok, 2, None) == 1          # unknown flag bit
     assert B.lib.lq_decode_step_ex(c, 128, 16, 16, 16, 16, 16, 16, 1, None) == 6
     assert B.lib.lq_decode_step_ex(c, None, 16, 16, 16, 16, 16, 16, 1, None) == 1
+
+
+def test_binding_checks_tensors_before_any_call(B, monkeypatch):
+    """The binding refuses a tensor of the wrong dtype, the wrong element count
+    or not on the current CUDA device, before the library is called (the C
+    side trusts the shapes it is given, so a bad buffer would otherwise be
+    read or written out of bounds on the GPU)."""
+    torch = pytest.importorskip("torch")
+    calls = []
+    real_lib = B.lib
+
+    class Spy:
+        def __getattr__(self, name):
+            real = getattr(real_lib, name)
+            if name == "lq_state_bytes":
+                return real
+            def f(*a):
+                calls.append(name)
+                return 0
+            return f
+
+    monkeypatch.setattr(B, "lib", Spy())
+    N, H, d = 2, 3, 64
+    cfg = B.make_config(N, H, d, d, bits=8, in_dtype="bf16")
+    nb = B.lq_state_bytes(cfg)
+    f32, bf16 = torch.float32, torch.bfloat16
+    good = dict(state=torch.zeros(N * H * nb, dtype=torch.uint8), q=torch.zeros(N, H, d, dtype=bf16),
+                k=torch.zeros(N, H, d, dtype=bf16), v=torch.zeros(N, H, d, dtype=bf16),
+                beta=torch.zeros(N, H, dtype=f32), decay=torch.zeros(N, H, dtype=f32),
+                out=torch.zeros(N, H, d, dtype=f32))
+
+    def step(**over):
+        a = {**good, **over}
+        B.lq_decode_step(cfg, a["state"], a["q"], a["k"], a["v"], a["beta"], a["decay"], a["out"], stream=0)
+
+    bad = [
+        ("dtype", dict(q=torch.zeros(N, H, d, dtype=f32))),
+        ("elements", dict(out=torch.zeros(N, H, d - 1, dtype=f32))),
+        ("elements", dict(decay=torch.zeros(N, H, d, dtype=f32))),   # KDA-sized decay on a GDN state
+        ("at least", dict(state=torch.zeros(N * H * nb - 1, dtype=torch.uint8))),
+    ]
+    for why, over in bad:
+        with pytest.raises(ValueError, match=why):
+            step(**over)
+    with pytest.raises(ValueError, match="CUDA tensor"):
+        step()                                   # right shapes and types, but host memory
+    with pytest.raises(ValueError, match="dtype"):
+        B.lq_state_init(cfg, good["state"], torch.zeros(N, H, d, d, dtype=torch.float64), stream=0)
+    with pytest.raises(ValueError, match="elements"):
+        B.lq_dequant_state(cfg, good["state"], torch.zeros(N, H, d, d + 1, dtype=f32), stream=0)
+    with pytest.raises(ValueError, match="dtype"):
+        B.lq_window_flush_slots(cfg, good["state"], torch.zeros(2, dtype=torch.int64), stream=0)
+    T = 3
+    with pytest.raises(ValueError, match="elements"):   # per-token tensors need T rows
+        B.lq_decode_steps(cfg, good["state"], T, good["q"], good["k"], good["v"], good["beta"],
+                          good["decay"], good["out"], stream=0)
+    with pytest.raises(ValueError, match="lengths"):
+        B.lq_prefill(cfg, good["state"], 1, good["q"], good["k"], good["v"], good["beta"], good["decay"],
+                     lengths=torch.zeros(N + 1, dtype=torch.int32), stream=0)
+    assert calls == []
+    # raw addresses are the caller's responsibility and pass through
+    B.lq_window_flush(cfg, 256, stream=0)
+    assert calls == ["lq_window_flush"]
