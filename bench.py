@@ -70,6 +70,14 @@ def parse_args():
     ap.add_argument("--no-slots", action="store_true",
                     help="skip the serving path (decode and flush through a slot list)")
     ap.add_argument("--cpu-seconds", type=float, default=10.0)
+    ap.add_argument("--no-configs", action="store_true",
+                    help="skip the per_config lines (KDA INT8, GDN 6-bit and 4-bit, the mixed sweep)")
+    ap.add_argument("--config-steps", type=int, default=40,
+                    help="timed window-steps of each per_config workload")
+    ap.add_argument("--sweep-tokens", type=int, default=4096,
+                    help="decode tokens of each point of the prefix-cache-scale sweep")
+    ap.add_argument("--sweep", default="8x2,8x4,8x8,16x2,16x4,16x8,32x2,32x4,32x8",
+                    help="WxR points of the prefix-cache-scale sweep (empty: skip it)")
     return ap.parse_args()
 
 
@@ -148,6 +156,21 @@ def fp32_bytes(wl):
     write the output."""
     f = field_bytes(wl)
     return 2 * 4 * wl.dk * wl.dv + f["inputs"] + f["out"]
+
+
+def restore_bytes(wl):
+    """A prefix-cache hit: the compact part of a flushed blob is read from the
+    pool and written into a live slot (algorithmic bytes per head; the copy
+    itself moves whole blobs)."""
+    f = field_bytes(wl)
+    compact = f["hdr"] + f["meta"] + f["qs"] + f["sm"] + f["cvec"] + f["codes"] + f["g"]
+    return 2 * compact
+
+
+def head_token_bytes(wl):
+    """Window-mean algorithmic bytes per head-token, the flush amortised."""
+    W = wl.window
+    return (sum(decode_bytes(wl, c) for c in range(W)) + flush_bytes(wl)) / W
 
 
 # ------------------------------------------------------------ helpers
@@ -515,6 +538,232 @@ def cpu_baseline(wl, layer_np, seconds, oracle):
                       f"{dt:.1f} s"}
 
 
+def measure_config(name, args, torch, B, I, hbm, dist, world):
+    """One more workload of the pages' setting, measured as the headline is:
+    the step (W decode tokens over L layer-states, then the flushes) and the
+    FP32-state kernel on the same inputs; L chosen so the rotated states are
+    far larger than L2."""
+    wl = rank_workload(I.WORKLOADS[name], int(os.environ.get("RANK", "0")))
+    nh = wl.batch * wl.heads
+    L = 4 if nh <= 4096 else 2
+    layers = make_layers(wl, L, torch, I)
+    arm = Arm(wl, layers, wl.bits, torch, B)
+    arm.capture()
+    ks = args.config_steps
+    total, dec, fl = time_arm(arm, ks, 3, torch, dist, world)
+    status = max(st.check() for st in arm.states)
+    if status != 0:
+        raise RuntimeError(f"device status after {name}: {B.STATUS_NAMES[status]}")
+    W = wl.window
+    value = whole_job_rate(ks * W * L * nh, world, total)
+    dec_ms = dec / (ks * W * L)
+    dbytes = nh * sum(decode_bytes(wl, c) for c in range(W)) / W
+    achieved = dbytes / (dec_ms / 1e3) / 1e9
+    step_bytes = nh * L * W * head_token_bytes(wl)
+    out = {"value": value, "unit": "head-tokens/s", "steps": ks, "layers_rotated": L,
+           "batch": wl.batch, "heads": wl.heads, "state_bits": wl.bits, "decay": wl.decay_kind,
+           "window": W, "num_comp": wl.num_comp, "scales": wl.scale_dtype,
+           "bytes_per_head_token": head_token_bytes(wl),
+           "roofline": {"bound": "hbm", "achieved": achieved, "peak": hbm, "unit": "GB/s",
+                        "frac": achieved / hbm, "kernel": f"decode_kernel<{wl.dk},{wl.bits}>",
+                        "algorithmic_bytes_per_launch": dbytes, "avg_launch_us": dec_ms * 1e3},
+           "step_frac": step_bytes / (total / ks / 1e3) / 1e9 / hbm,
+           "flush_avg_launch_us": fl / (ks * L) * 1e3}
+    del arm
+    torch.cuda.empty_cache()
+    arm32 = Arm(wl, layers, 32, torch, B)
+    arm32.capture()
+    t32, d32, _ = time_arm(arm32, max(4, ks // 2), 3, torch, dist, world)
+    v32 = whole_job_rate(max(4, ks // 2) * W * L * nh, world, t32)
+    a32 = nh * fp32_bytes(wl) / (d32 / (max(4, ks // 2) * W * L) / 1e3) / 1e9
+    out["fp32_state"] = {"value": v32, "achieved_gbs": a32, "frac": a32 / hbm}
+    out["vs_fp32_state_kernel"] = value / v32
+    del arm32, layers
+    torch.cuda.empty_cache()
+    return out
+
+
+class MixedLayer:
+    """The prefix-cache-scale layer: 48 heads per sequence, held as a GDN state
+    (36 heads) and a KDA state (12 heads), B live sequences, plus a pool of
+    cached flushed sequences that are restored into live slots (prefix-cache
+    hits, lq_copy_slots) at window boundaries, spread evenly over the run."""
+
+    def __init__(self, wls, S0s, devs, pool_slots, torch, B, bits=8):
+        self.wls, self.torch, self.B = wls, torch, B
+        self.W = wls[0].window
+        self.states, self.pools, self.inp, self.out, self.cfgs = [], [], [], [], []
+        for wl, S0, dev in zip(wls, S0s, devs):
+            cfg = B.config_for(wl, bits=bits)
+            st = B.LQState(cfg)
+            st.init(S0)
+            pcfg = B.config_for(wl, bits=bits)
+            pcfg.num_slots = pool_slots
+            pool = B.LQState(pcfg)
+            for h in range(0, pool_slots, wl.batch):   # the pool holds flushed entries
+                n = min(wl.batch, pool_slots - h)
+                sl = torch.arange(h, h + n, dtype=torch.int32, device="cuda")
+                pool.init_slots(sl, S0[:n].contiguous())
+            self.cfgs.append(cfg)
+            self.states.append(st)
+            self.pools.append(pool)
+            self.inp.append({k: v[:self.W] for k, v in dev.items()})
+            self.out.append(torch.empty((self.W, wl.batch, wl.heads, wl.dv), dtype=torch.float32,
+                                        device="cuda"))
+        self.flags = B.LQ_STEP_EARLY_STATE
+        torch.cuda.synchronize()
+
+    def decode_all(self):
+        for t in range(self.W):
+            for l, st in enumerate(self.states):
+                x = self.inp[l]
+                st.step(x["q"][t], x["k"][t], x["v"][t], x["beta"][t], x["decay"][t], self.out[l][t],
+                        flags=self.flags)
+
+    def flush_all(self):
+        for st in self.states:
+            st.flush()
+
+    def restore(self, dst, src):
+        """Cached pool entries src -> live slots dst (both int32 device lists),
+        after the window's flushes; a plain launch, so the next step's early
+        staging never overlaps it."""
+        B = self.B
+        for l, st in enumerate(self.states):
+            pool = self.pools[l]
+            B.lq_copy_slots(self.cfgs[l], st.buf, self.cfgs[l].num_slots, dst, pool.buf,
+                            pool.cfg.num_slots, src)
+
+
+def measure_sweep(args, torch, B, I, hbm, dist, world):
+    """Config 4: W x r sweep of the mixed 3:1 GDN:KDA layer at 512 live
+    sequences, with 1024 cached INT8 sequences restored once each over the
+    run (one hit per four tokens)."""
+    points = [tuple(int(x) for x in p.split("x")) for p in args.sweep.split(",") if p]
+    if not points:
+        return None
+    rank = int(os.environ.get("RANK", "0"))
+    base = [rank_workload(I.WORKLOADS[n], rank) for n in ("mix_gdn_b512h36", "mix_kda_b512h12")]
+    Wmax = max(W for W, _ in points)
+    S0s, devs = [], []
+    for wl in base:
+        s = I.InputStream(wl, stream=0)
+        st = s.state()
+        S0s.append(torch.from_numpy(st["S0"]).cuda())
+        del st
+        devs.append(I.to_device(wl, s.tokens(Wmax)))
+    pool_slots = 1024
+    live = base[0].batch
+    nh = sum(wl.batch * wl.heads for wl in base)
+    res = {"layer": "48 heads per sequence: 36 GDN + 12 KDA (two states)", "live_slots": live,
+           "cached_sequences": pool_slots, "tokens_per_point": args.sweep_tokens,
+           "hits": "one cached sequence restored per 4 tokens, cycling through the pool", "points": {}}
+    E = torch.cuda.Event
+    for W, r in points:
+        wls = [wl.replace(window=W, num_comp=r) for wl in base]
+        layer = MixedLayer(wls, S0s, devs, pool_slots, torch, B)
+        steps = max(1, args.sweep_tokens // W)
+        hits_per_step = max(1, W // 4)
+        n_hits = steps * hits_per_step
+        dst_all = torch.tensor([(i * 37) % live for i in range(n_hits)], dtype=torch.int32, device="cuda")
+        src_all = torch.tensor([i % pool_slots for i in range(n_hits)], dtype=torch.int32, device="cuda")
+        layer.decode_all()
+        layer.flush_all()
+        torch.cuda.synchronize()
+        sgraph = torch.cuda.Stream()
+        sgraph.wait_stream(torch.cuda.current_stream())
+        g_dec, g_fl = torch.cuda.CUDAGraph(), torch.cuda.CUDAGraph()
+        with torch.cuda.graph(g_dec, stream=sgraph):
+            layer.decode_all()
+        with torch.cuda.graph(g_fl, stream=sgraph):
+            layer.flush_all()
+        torch.cuda.synchronize()
+        for x in range(2):  # warm-up windows (with restores of the first entries)
+            g_dec.replay()
+            g_fl.replay()
+            layer.restore(dst_all[:hits_per_step], src_all[:hits_per_step])
+        torch.cuda.synchronize()
+        marks = [(E(enable_timing=True), E(enable_timing=True), E(enable_timing=True)) for _ in range(steps)]
+        a, b = E(enable_timing=True), E(enable_timing=True)
+        if world > 1:
+            dist.barrier()
+        torch.cuda.synchronize()
+        a.record()
+        for sidx in range(steps):
+            m0, m1, m2 = marks[sidx]
+            m0.record()
+            g_dec.replay()
+            m1.record()
+            g_fl.replay()
+            m2.record()
+            h0 = sidx * hits_per_step
+            layer.restore(dst_all[h0:h0 + hits_per_step], src_all[h0:h0 + hits_per_step])
+        b.record()
+        torch.cuda.synchronize()
+        total = a.elapsed_time(b)
+        dec = sum(x.elapsed_time(y) for x, y, _ in marks)
+        fl = sum(y.elapsed_time(z) for _, y, z in marks)
+        total, dec, fl = max_over_ranks([total, dec, fl], torch, dist, world, "cuda")
+        status = max(st.check() for st in layer.states)
+        if status != 0:
+            raise RuntimeError(f"device status after sweep point W={W} r={r}: {B.STATUS_NAMES[status]}")
+        tok = steps * W
+        per_ht = sum(wl.batch * wl.heads * head_token_bytes(wl) for wl in wls) / nh
+        per_ht += sum(n_hits * wl.heads * restore_bytes(wl) for wl in wls) / (nh * tok)
+        dbytes = sum(wl.batch * wl.heads * sum(decode_bytes(wl, c) for c in range(W)) for wl in wls) / W
+        dec_us = dec / (steps * W) * 1e3   # both states' decode launches of one token
+        res["points"][f"W{W}_r{r}"] = {
+            "value": whole_job_rate(tok * nh, world, total), "unit": "head-tokens/s",
+            "steps": steps, "hits": n_hits, "bytes_per_head_token": per_ht,
+            "step_frac": per_ht * tok * nh / (total / 1e3) / 1e9 / hbm,
+            "decode_frac": dbytes / (dec_us / 1e6) / 1e9 / hbm,
+            "decode_us_per_token": dec_us, "flush_us_per_window": fl / steps * 1e3}
+        del layer, g_dec, g_fl
+        torch.cuda.empty_cache()
+    # the FP32-state kernel on the same 48-head layer (independent of W and r)
+    v32 = None
+    states32 = []
+    for wl, S0 in zip(base, S0s):
+        st = B.LQState(B.config_for(wl, bits=32))
+        st.init(S0)
+        states32.append(st)
+    ins = [{k: v[:16] for k, v in d.items()} for d in devs]
+    outs = [torch.empty((16, wl.batch, wl.heads, wl.dv), dtype=torch.float32, device="cuda") for wl in base]
+
+    def fp32_window():
+        for t in range(16):
+            for l, st in enumerate(states32):
+                x = ins[l]
+                st.step(x["q"][t], x["k"][t], x["v"][t], x["beta"][t], x["decay"][t], outs[l][t])
+
+    fp32_window()
+    torch.cuda.synchronize()
+    g32 = torch.cuda.CUDAGraph()
+    sg = torch.cuda.Stream()
+    sg.wait_stream(torch.cuda.current_stream())
+    with torch.cuda.graph(g32, stream=sg):
+        fp32_window()
+    for _ in range(2):
+        g32.replay()
+    torch.cuda.synchronize()
+    k32 = 8
+    a, b = E(enable_timing=True), E(enable_timing=True)
+    a.record()
+    for _ in range(k32):
+        g32.replay()
+    b.record()
+    torch.cuda.synchronize()
+    ms32 = max_over_ranks([a.elapsed_time(b)], torch, dist, world, "cuda")[0]
+    v32 = whole_job_rate(k32 * 16 * nh, world, ms32)
+    res["fp32_state"] = {"value": v32, "unit": "head-tokens/s",
+                         "frac": nh * fp32_bytes(base[0]) * k32 * 16 / (ms32 / 1e3) / 1e9 / hbm}
+    for p in res["points"].values():
+        p["vs_fp32_state_kernel"] = p["value"] / v32
+    del states32, g32, S0s, devs
+    torch.cuda.empty_cache()
+    return res
+
+
 def config_of(wl, args, world):
     return {"workload": wl.name, "batch": wl.batch, "heads": wl.heads, "dk": wl.dk, "dv": wl.dv,
             "window": wl.window, "num_comp": wl.num_comp, "state_bits": wl.bits,
@@ -714,6 +963,16 @@ def main_ours(args):
             "flush_avg_launch_us": fs / (kss * L) * 1e3}
         del arms
         torch.cuda.empty_cache()
+
+    # ---- the other workloads of the pages' setting, each on its own
+    if not args.no_configs:
+        pc = {}
+        for name in ("kda_int8_b128h32", "gdn_6bit_b256h32", "gdn_4bit_b256h32"):
+            pc[name] = measure_config(name, args, torch, B, I, hbm, dist, world)
+        sweep = measure_sweep(args, torch, B, I, hbm, dist, world)
+        if sweep is not None:
+            pc["mix_b512h48_sweep"] = sweep
+        line["per_config"] = pc
 
     # ---- end to end through the public calls with host buffers
     if not args.no_e2e:

@@ -77,3 +77,11 @@ def test_state_memory_figures(bench, wl):
     assert m["fp32_blob_bytes"] >= 4 * 128 * 128
     assert 3.0 < m["compact_vs_fp32"] < 3.5
     assert m["layer_leapquant_mb"] == 2048 * 36096 / 1e6
+
+
+def test_head_token_bytes_and_restore_bytes(bench, wl):
+    # window mean of the decode bytes plus the flush spread over the window
+    assert bench.head_token_bytes(wl) == (29492 * 16 + 55364) / 16
+    # a prefix-cache hit reads and writes the compact part: header 20, meta 16,
+    # qs 512, sm 512, compensators 2048, codes 16384
+    assert bench.restore_bytes(wl) == 2 * (20 + 16 + 512 + 512 + 2048 + 16384)
