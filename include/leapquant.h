@@ -220,8 +220,9 @@ LQ_API lq_status lq_check_status(const lq_config *cfg, const void *state, lq_str
  *      the previous kernel is, say, the projection that produces q, k, v;
  *      false when two steps on the same state follow each other directly.  A
  *      wrong promise reads stale state.
- * Other bits: LQ_ERR_INVALID_ARG.  The flag changes nothing for bits = 32
- * and per_step states. */
+ * Other bits: LQ_ERR_INVALID_ARG.  The flag applies to every format: for
+ * bits = 32 and the per_step states the dense state of the first heads is
+ * staged early in the same way. */
 #define LQ_STEP_EARLY_STATE 0x1u
 LQ_API lq_status lq_decode_step_ex(const lq_config *cfg, void *state, const void *q, const void *k,
                                    const void *v, const float *beta, const float *decay, float *out,

@@ -10,6 +10,7 @@
 #include "leapquant.h"
 #include "lq_common.cuh"
 #include "lq_decode.cuh"
+#include "lq_dense.cuh"
 #include "lq_flush.cuh"
 #include "lq_fp32.cuh"
 #include "lq_perstep.cuh"
@@ -178,10 +179,29 @@ lq_status dispatch_decode(const lq_config &c, const DecodeArgs &a, cudaStream_t 
     }
 }
 
-template <int D>
-lq_status launch_fp32_decode(const lq_config &c, const Fp32Args &a, cudaStream_t s) {
-    const int grid = a.num_heads * (D / kFp32Cols);
-    return launched(launch_pdl(fp32_decode_kernel<D>, grid, kFp32Threads, 0u, s, a));
+// The dense decode step (FP32 state, or a per-step BF16 / FP8 state):
+// persistent, one CTA per SM (the stage ring takes most of shared memory).
+template <int D, int FMT>
+lq_status launch_dense_step(const DenseArgs &a, cudaStream_t s) {
+    const uint32_t smem = dense_smem_bytes(D, FMT, a.F.bf16_in, a.F.kda);
+    auto k = dense_step_kernel<D, FMT>;
+    if (allow_smem(k, smem) != cudaSuccess) return LQ_ERR_CUDA;
+    const int grid = persistent_grid(k, DenseShape<D>::NT, smem, a.num_heads);
+    if (grid <= 0) return LQ_ERR_CUDA;
+    return launched(launch_pdl(k, grid, DenseShape<D>::NT, smem, s, a));
+}
+
+lq_status dispatch_dense_step(const lq_config &c, const DenseArgs &a, cudaStream_t s) {
+    const int fmt = c.per_step ? c.bits : 32;
+    switch (c.dk * 100 + fmt) {
+        case 12832: return launch_dense_step<128, 32>(a, s);
+        case 12816: return launch_dense_step<128, 16>(a, s);
+        case 12808: return launch_dense_step<128, 8>(a, s);
+        case 6432: return launch_dense_step<64, 32>(a, s);
+        case 6416: return launch_dense_step<64, 16>(a, s);
+        case 6408: return launch_dense_step<64, 8>(a, s);
+        default: return LQ_ERR_UNSUPPORTED;
+    }
 }
 
 // The per-step baselines: one 128-thread CTA per (slot, head) and 64-column
@@ -334,15 +354,10 @@ lq_status lq_decode_step_ex(const lq_config *cfg, void *state, const void *q, co
     const lq_config &c = *cfg;
     const Layout L = make_layout(c);
     cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
-    if (c.per_step) {
-        Fp32Args a{static_cast<uint8_t *>(state), nullptr, nullptr, L, make_flags(c), q, k, v,
-                   beta, decay, out, c.num_slots * c.num_heads};
-        return dispatch_perstep<0>(c, a, s);
-    }
-    if (c.bits == 32) {
-        Fp32Args a{static_cast<uint8_t *>(state), nullptr, nullptr, L, make_flags(c), q, k, v,
-                   beta, decay, out, c.num_slots * c.num_heads};
-        return c.dk == 128 ? launch_fp32_decode<128>(c, a, s) : launch_fp32_decode<64>(c, a, s);
+    if (c.per_step || c.bits == 32) {
+        DenseArgs a{static_cast<uint8_t *>(state), L, make_flags(c), q, k, v, beta, decay, out,
+                    c.num_slots * c.num_heads, flags};
+        return dispatch_dense_step(c, a, s);
     }
     DecodeArgs a{static_cast<uint8_t *>(state), L, make_flags(c), q, k, v, beta, decay, out,
                  c.num_slots * c.num_heads, SlotMap{nullptr, c.num_heads, c.num_slots}, 1, flags};

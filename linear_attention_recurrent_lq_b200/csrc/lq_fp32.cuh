@@ -1,17 +1,7 @@
-// lq_fp32.cuh -- the FP32-state reference path (bits = 32): every decode
-// token reads the dense FP32 state of each head from HBM, updates it and
-// writes it back.  This is the cost LeapQuant removes (news post "Linear
-// attention has to move state every token it generates; LeapQuant
-// compresses it to 8-bit without losing accuracy", second paragraph); the
-// library keeps it as the comparison point for throughput and accuracy.
-//
-// The update separates by value column: u_j = beta (v_j - (S'^T k)_j) needs
-// only column j of S' = D_t S.  So one CTA of 128 threads takes one
-// (slot, head) and a block of 32 value columns: thread t loads rows
-// TI*(t%16).. (TI = D/16) of columns 4*(t/16).. of the block straight into
-// registers with 16-byte loads, forms S', the column sums S'^T k and S'^T q
-// meet in shared memory, and it writes S' + k u^T back with 16-byte stores.
-// Many small CTAs per SM keep the loads of several heads in flight.
+// lq_fp32.cuh -- entering and reading back the FP32-state reference path
+// (bits = 32): the state is stored as it is, so init copies S0 into the
+// blobs and read-back copies it out.  The decode step of this path (and of
+// the per-step baselines) is dense_step_kernel in lq_dense.cuh.
 #pragma once
 
 #include "lq_common.cuh"
@@ -32,90 +22,6 @@ struct Fp32Args {
     float *out;
     int num_heads;
 };
-
-template <int D>
-__global__ void __launch_bounds__(kFp32Threads) fp32_decode_kernel(Fp32Args A) {
-    constexpr int TI = D / 16, NB = D / kFp32Cols;
-    pdl_wait();
-    pdl_trigger();
-    const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
-    const int ic = tid & 15, jc = tid >> 4, i0 = TI * ic;
-    const size_t head = blockIdx.x / NB;
-    const int cb = blockIdx.x % NB, j0 = kFp32Cols * cb + 4 * jc;
-    const Flags &F = A.F;
-    uint8_t *blob = A.state + head * A.L.blob;
-    float *S = reinterpret_cast<float *>(blob + kHdrBytes);
-
-    __shared__ float s_pk[16][kFp32Cols], s_pq[16][kFp32Cols], s_u[kFp32Cols], s_kq[kFp32Threads / 32];
-
-    const uint4 hdr = *reinterpret_cast<const uint4 *>(blob);
-    const bool run = hdr.w == kMagic && hdr.y == 0;
-    if (!run) {
-        if (tid < kFp32Cols) A.out[head * D + kFp32Cols * cb + tid] = 0.f;
-        if (hdr.w != kMagic && hdr.y == 0 && cb == 0 && tid == 0) set_status(blob, LQ_DEV_CORRUPT);
-        return;
-    }
-    float4 r4[TI];
-#pragma unroll
-    for (int ii = 0; ii < TI; ++ii) r4[ii] = __ldcs(reinterpret_cast<const float4 *>(S + (size_t)(i0 + ii) * D + j0));
-    float kr[TI], qr[TI], ar[TI];
-#pragma unroll
-    for (int ii = 0; ii < TI; ++ii) {
-        const size_t o = head * D + i0 + ii;
-        kr[ii] = load_in(A.k, o, F.bf16_in);
-        qr[ii] = load_in(A.q, o, F.bf16_in);
-        ar[ii] = F.kda ? A.decay[o] : A.decay[head];
-    }
-    float kq = 0.f;
-    if (tid < D) {
-        const size_t o = head * D + tid;
-        kq = load_in(A.k, o, F.bf16_in) * load_in(A.q, o, F.bf16_in);
-    }
-#pragma unroll
-    for (int off = 16; off >= 1; off >>= 1) kq += __shfl_xor_sync(0xFFFFFFFFu, kq, off);
-    if (lane == 0) s_kq[warp] = kq;
-
-    float Sd[TI][4];
-    float pk[4] = {0.f, 0.f, 0.f, 0.f}, pq[4] = {0.f, 0.f, 0.f, 0.f};
-#pragma unroll
-    for (int ii = 0; ii < TI; ++ii) {
-        const float a = ar[ii];
-        Sd[ii][0] = a * r4[ii].x; Sd[ii][1] = a * r4[ii].y; Sd[ii][2] = a * r4[ii].z; Sd[ii][3] = a * r4[ii].w;
-#pragma unroll
-        for (int jj = 0; jj < 4; ++jj) {
-            pk[jj] = fmaf(Sd[ii][jj], kr[ii], pk[jj]);
-            pq[jj] = fmaf(Sd[ii][jj], qr[ii], pq[jj]);
-        }
-    }
-    *reinterpret_cast<float4 *>(&s_pk[ic][4 * jc]) = make_float4(pk[0], pk[1], pk[2], pk[3]);
-    *reinterpret_cast<float4 *>(&s_pq[ic][4 * jc]) = make_float4(pq[0], pq[1], pq[2], pq[3]);
-    __syncthreads();
-    if (tid < kFp32Cols) {
-        float a = 0.f, b = 0.f, kq_all = 0.f;
-#pragma unroll
-        for (int r = 0; r < 16; ++r) {
-            a += s_pk[r][tid];
-            b += s_pq[r][tid];
-        }
-#pragma unroll
-        for (int w = 0; w < kFp32Threads / 32; ++w) kq_all += s_kq[w];
-        const size_t o = head * D + kFp32Cols * cb + tid;
-        const float u = A.beta[head] * (load_in(A.v, o, F.bf16_in) - a);
-        s_u[tid] = u;
-        A.out[o] = fmaf(kq_all, u, b);
-    }
-    __syncthreads();
-    const float4 u4 = *reinterpret_cast<const float4 *>(&s_u[4 * jc]);
-#pragma unroll
-    for (int ii = 0; ii < TI; ++ii) {
-        float4 o4;
-        o4.x = fmaf(kr[ii], u4.x, Sd[ii][0]);
-        o4.y = fmaf(kr[ii], u4.y, Sd[ii][1]);
-        o4.z = fmaf(kr[ii], u4.z, Sd[ii][2]);
-        o4.w = fmaf(kr[ii], u4.w, Sd[ii][3]);
-        __stcs(reinterpret_cast<float4 *>(S + (size_t)(i0 + ii) * D + j0), o4);
-    }
-}
 
 template <int D, int MODE>
 __global__ void __launch_bounds__(256) fp32_copy_kernel(Fp32Args A) {

@@ -1,24 +1,19 @@
-// lq_perstep.cuh -- the naive per-step baselines: a dense state stored in
-// BF16, or in FP8 E4M3 with one FP32 scale per value column, rounded again
-// after every token.  These are the comparison points of the accuracy table
-// of the news post "Linear attention has to move state every token it
-// generates; LeapQuant compresses it to 8-bit without losing accuracy" (its
-// BF16 and FP8 rows): quantizing at every step lets the rounding error
-// compound, which LeapQuant's per-window scheme avoids.
-//
-// Same decomposition as the FP32-state kernel: the update separates by value
-// column, so one CTA of 128 threads takes one (slot, head) and a block of 64
-// value columns; thread t owns rows TI*(t%16).. (TI = D/16) of columns
-// 8*(t/16).. of the block (16-byte BF16 / 8-byte FP8 row segments).  The state is read and converted to FP32, the FP32
-// delta-rule step runs as in that kernel, and the new FP32 values are stored
-// back in the narrow format:
+// lq_perstep.cuh -- entering and reading back the naive per-step baselines:
+// a dense state stored in BF16, or in FP8 E4M3 with one FP32 scale per value
+// column (the BF16 and FP8 rows of the accuracy table of the news post
+// "Linear attention has to move state every token it generates; LeapQuant
+// compresses it to 8-bit without losing accuracy": quantizing at every step
+// lets the rounding error compound, which LeapQuant's per-window scheme
+// avoids).  The decode step of these formats is dense_step_kernel
+// (lq_dense.cuh), which rounds the same way:
 //  * BF16: each entry rounded to bfloat16, ties to even;
-//  * FP8: the column maxima meet in shared memory, scale_j =
-//    fl32(max_i |S_ij| / 448), code = E4M3(fl32(S_ij / scale_j)) with ties to
-//    even and saturation at 448 (an all-zero column: scale 0, codes 0); the
-//    value read back is fl32(E4M3 value * scale_j).
-// MODE 0 is the decode step, MODE 1 stores a caller's FP32 state (entering a
-// sequence), MODE 2 writes the dense FP32 values back out.
+//  * FP8: scale_j = fl32(max_i |S_ij| / 448), code = E4M3(fl32(S_ij /
+//    scale_j)) with ties to even and saturation at 448 (an all-zero column:
+//    scale 0, codes 0); the value read back is fl32(E4M3 value * scale_j).
+// One CTA of 128 threads per (slot, head) and block of 64 value columns;
+// thread t owns rows TI*(t%16).. (TI = D/16) of columns 8*(t/16).. of the
+// block.  MODE 1 stores a caller's FP32 state (entering a sequence), MODE 2
+// writes the dense FP32 values back out.
 #pragma once
 
 #include <cuda_bf16.h>
@@ -41,18 +36,17 @@ template <int D, int FMT, int MODE>
 __global__ void __launch_bounds__(kFp32Threads) perstep_kernel(Fp32Args A) {
     constexpr int TI = D / 16, NB = D / kPsCols, CPT = kPsCpt;
     static_assert(FMT == 16 || FMT == 8, "BF16 or FP8 state");
+    static_assert(MODE == 1 || MODE == 2, "init or read-back");
     pdl_wait();
     pdl_trigger();
-    const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
+    const int tid = threadIdx.x;
     const int ic = tid & 15, jc = tid >> 4, i0 = TI * ic;
     const size_t head = blockIdx.x / NB;
     const int cb = blockIdx.x % NB, j0 = kPsCols * cb + CPT * jc;
-    const Flags &F = A.F;
     const Layout &L = A.L;
     uint8_t *blob = A.state + head * L.blob;
 
-    __shared__ float s_pk[16][kPsCols], s_pq[16][kPsCols], s_u[kPsCols], s_sc[kPsCols];
-    __shared__ float s_kq[kFp32Threads / 32];
+    __shared__ float s_pk[16][kPsCols], s_sc[kPsCols];
 
     // ---- the current state in FP32
     float Sd[TI][CPT];
@@ -66,14 +60,6 @@ __global__ void __launch_bounds__(kFp32Threads) perstep_kernel(Fp32Args A) {
             Sd[ii][4] = b4.x; Sd[ii][5] = b4.y; Sd[ii][6] = b4.z; Sd[ii][7] = b4.w;
         }
     } else {
-        if constexpr (MODE == 0) {
-            const uint4 hdr = *reinterpret_cast<const uint4 *>(blob);
-            if (!(hdr.w == kMagic && hdr.y == 0)) {
-                if (tid < kPsCols) A.out[head * D + kPsCols * cb + tid] = 0.f;
-                if (hdr.w != kMagic && hdr.y == 0 && cb == 0 && tid == 0) set_status(blob, LQ_DEV_CORRUPT);
-                return;
-            }
-        }
         if constexpr (FMT == 16) {
             const uint16_t *Sb = reinterpret_cast<const uint16_t *>(blob + L.codes_off);
 #pragma unroll
@@ -109,66 +95,6 @@ __global__ void __launch_bounds__(kFp32Threads) perstep_kernel(Fp32Args A) {
             *reinterpret_cast<float4 *>(row + 4) = make_float4(Sd[ii][4], Sd[ii][5], Sd[ii][6], Sd[ii][7]);
         }
         return;
-    }
-
-    // ---- MODE 0: the FP32 delta-rule step (as in the FP32-state kernel)
-    if constexpr (MODE == 0) {
-        float kr[TI], qr[TI];
-#pragma unroll
-        for (int ii = 0; ii < TI; ++ii) {
-            const size_t o = head * D + i0 + ii;
-            kr[ii] = load_in(A.k, o, F.bf16_in);
-            qr[ii] = load_in(A.q, o, F.bf16_in);
-            const float a = F.kda ? A.decay[o] : A.decay[head];
-#pragma unroll
-            for (int jj = 0; jj < CPT; ++jj) Sd[ii][jj] = a * Sd[ii][jj];
-        }
-        float kq = 0.f;
-        if (tid < D) {
-            const size_t o = head * D + tid;
-            kq = load_in(A.k, o, F.bf16_in) * load_in(A.q, o, F.bf16_in);
-        }
-#pragma unroll
-        for (int off = 16; off >= 1; off >>= 1) kq += __shfl_xor_sync(0xFFFFFFFFu, kq, off);
-        if (lane == 0) s_kq[warp] = kq;
-        float pk[CPT], pq[CPT];
-#pragma unroll
-        for (int jj = 0; jj < CPT; ++jj) pk[jj] = pq[jj] = 0.f;
-#pragma unroll
-        for (int ii = 0; ii < TI; ++ii)
-#pragma unroll
-            for (int jj = 0; jj < CPT; ++jj) {
-                pk[jj] = fmaf(Sd[ii][jj], kr[ii], pk[jj]);
-                pq[jj] = fmaf(Sd[ii][jj], qr[ii], pq[jj]);
-            }
-#pragma unroll
-        for (int jj = 0; jj < CPT; ++jj) {
-            s_pk[ic][CPT * jc + jj] = pk[jj];
-            s_pq[ic][CPT * jc + jj] = pq[jj];
-        }
-        __syncthreads();
-        if (tid < kPsCols) {
-            float a = 0.f, b = 0.f, kq_all = 0.f;
-#pragma unroll
-            for (int r = 0; r < 16; ++r) {
-                a += s_pk[r][tid];
-                b += s_pq[r][tid];
-            }
-#pragma unroll
-            for (int w = 0; w < kFp32Threads / 32; ++w) kq_all += s_kq[w];
-            const size_t o = head * D + kPsCols * cb + tid;
-            const float u = A.beta[head] * (load_in(A.v, o, F.bf16_in) - a);
-            s_u[tid] = u;
-            A.out[o] = fmaf(kq_all, u, b);
-        }
-        __syncthreads();
-        float uu[CPT];
-#pragma unroll
-        for (int jj = 0; jj < CPT; ++jj) uu[jj] = s_u[CPT * jc + jj];
-#pragma unroll
-        for (int ii = 0; ii < TI; ++ii)
-#pragma unroll
-            for (int jj = 0; jj < CPT; ++jj) Sd[ii][jj] = fmaf(kr[ii], uu[jj], Sd[ii][jj]);
     }
 
     // ---- store the new FP32 values in the narrow format

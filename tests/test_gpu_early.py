@@ -1,7 +1,8 @@
 """The early-state flag of lq_decode_step_ex: with states taking turns on
 the stream (the previous launch never writes the next one's state), a
 window of flagged steps and its flush give, bit for bit, the outputs and
-blobs of unflagged steps."""
+blobs of unflagged steps; for the LeapQuant formats, the FP32-state
+reference and the per-step BF16 / FP8 baselines."""
 import pytest
 
 from linear_attention_recurrent_lq_b200 import inputs as I
@@ -21,16 +22,21 @@ def _cuda():
     build.build()
 
 
-@pytest.mark.parametrize("kind,bits", [("gdn_int8_b64h32", 8), ("kda_int8_b128h32", 4),
-                                       ("gdn_int8_b64h32", 6)])
-def test_early_state_steps_equal_plain_steps(kind, bits):
+@pytest.mark.parametrize("kind,bits,per_step", [("gdn_int8_b64h32", 8, False), ("kda_int8_b128h32", 4, False),
+                                                ("gdn_int8_b64h32", 6, False), ("gdn_int8_b64h32", 32, False),
+                                                ("kda_int8_b128h32", 32, False), ("gdn_int8_b64h32", 16, True),
+                                                ("kda_int8_b128h32", 8, True)])
+def test_early_state_steps_equal_plain_steps(kind, bits, per_step):
     from linear_attention_recurrent_lq_b200 import binding as B
-    wl = I.WORKLOADS[kind].replace(batch=7, heads=9, window=8)  # 63 heads: several per CTA
+    # 63 heads: several per CTA of the LeapQuant decode; with 1200 heads the
+    # dense kernels (one CTA per SM) walk several heads per CTA as well
+    wl = I.WORKLOADS[kind].replace(batch=7 if bits in (8, 6, 4) and not per_step else 40,
+                                   heads=9 if bits in (8, 6, 4) and not per_step else 30, window=8)
     L, T = 3, 12  # three layer-states taking turns; a flush after token 8
     draws = [I.InputStream(wl, stream=l) for l in range(L)]
     st0 = [s.state() for s in draws]
     toks = [s.tokens(T) for s in draws]
-    cfg = B.config_for(wl, bits=bits)
+    cfg = B.config_for(wl, bits=bits, per_step=per_step)
     plain, early = [], []
     for l in range(L):
         for group in (plain, early):
