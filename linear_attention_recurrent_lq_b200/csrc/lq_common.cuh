@@ -39,7 +39,7 @@ struct Layout {
     uint32_t scale_bytes;    // 4 (f32) or 2 (f16)
 };
 
-__host__ __device__ inline uint32_t align_up(uint32_t x, uint32_t a) { return (x + a - 1) / a * a; }
+__host__ __device__ constexpr uint32_t align_up(uint32_t x, uint32_t a) { return (x + a - 1) / a * a; }
 
 inline Layout make_layout(const lq_config &c) {
     Layout L{};

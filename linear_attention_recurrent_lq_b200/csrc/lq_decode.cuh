@@ -432,6 +432,22 @@ __global__ void __launch_bounds__(D + 64, (SLOTS || MULTI) ? 3 : 0) decode_kerne
 
     if (warp == COPY_WARP) {
         // ------------------------------------------------ copy warp
+        // Early instance: the token's inputs of the two staged heads go out at
+        // once, so their latency overlaps the reads of the window counts,
+        // beta and the decays below (the stages complete with the arrivals
+        // in the loop).
+        if (EARLY && lane == 0)
+            for (int x = 0; x < kDecodeStages && x < n_mine; ++x) {
+                const size_t h = blockIdx.x + (size_t)x * G;
+                uint8_t *st = stages + (size_t)x * SG.bytes;
+                mbar_expect_tx(&full[x], 3 * SG.qkv_bytes + (F.kda ? (uint32_t)D * 4u : 0u));
+                const size_t qo = h * (size_t)SG.qkv_bytes;
+                bulk_g2s(st + SG.in_off, static_cast<const uint8_t *>(A.q) + qo, SG.qkv_bytes, &full[x]);
+                bulk_g2s(st + SG.in_off + SG.qkv_bytes, static_cast<const uint8_t *>(A.k) + qo, SG.qkv_bytes, &full[x]);
+                bulk_g2s(st + SG.in_off + 2 * SG.qkv_bytes, static_cast<const uint8_t *>(A.v) + qo, SG.qkv_bytes,
+                         &full[x]);
+                if (F.kda) bulk_g2s(st + SG.dec_off, A.decay + h * D, (uint32_t)D * 4u, &full[x]);
+            }
         for (int base = 0; base < n_mine; base += 32) {
             const int i = base + lane;
             if (i < n_mine) {
@@ -483,7 +499,8 @@ __global__ void __launch_bounds__(D + 64, (SLOTS || MULTI) ? 3 : 0) decode_kerne
                     const uint8_t *blob = A.state + (size_t)s_bidx[x] * L.blob;
                     const uint32_t in_bytes = (uint32_t)T * (3 * SG.qkv_bytes + (F.kda ? (uint32_t)D * 4u : 0u));
                     if (EARLY && it < kDecodeStages) {
-                        mbar_arrive_expect_tx(&full[s], in_bytes);  // the state is on its way already
+                        mbar_arrive(&full[s]);  // state and inputs are on their way already
+                        continue;
                     } else {
                         const uint32_t cnt = s_cnt[x];
                         const uint32_t cc = cnt < (uint32_t)F.window ? cnt : 0u;
