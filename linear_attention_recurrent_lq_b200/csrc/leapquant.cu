@@ -15,6 +15,7 @@
 #include "lq_fp32.cuh"
 #include "lq_perstep.cuh"
 #include "lq_prefill.cuh"
+#include "lq_chunked.cuh"
 
 using namespace lq;
 
@@ -258,6 +259,12 @@ lq_status check_slots(const lq_config *cfg, const void *state, const int32_t *sl
 
 template <int D, int BITS>
 lq_status launch_prefill(const PrefillArgs &a, cudaStream_t s) {
+    if constexpr (D == 128) {  // the chunkwise form on the tensor cores
+        const uint32_t smem = chunk_prefill_smem_bytes(a.F);
+        auto k = a.map.slots ? chunk_prefill_kernel<BITS, true> : chunk_prefill_kernel<BITS, false>;
+        if (allow_smem(k, smem) != cudaSuccess) return LQ_ERR_CUDA;
+        return launched(launch_pdl(k, a.num_heads, kGroup, smem, s, a));
+    }
     const uint32_t smem = prefill_smem_bytes(D, BITS, a.F);
     auto k = a.map.slots ? prefill_kernel<D, BITS, true> : prefill_kernel<D, BITS, false>;
     if (allow_smem(k, smem) != cudaSuccess) return LQ_ERR_CUDA;
