@@ -933,15 +933,23 @@ def main_ours(args):
         status = stp.check()
         if status != 0:
             raise RuntimeError(f"device status after prefill: {B.STATUS_NAMES[status]}")
-        # FP32 work per head-token: decay (1), S'^T k and S'^T q (2 x 2), update (2) flops per entry
-        flops = 7.0 * wl.dk * wl.dv * nh * Tp
-        sms = props.multi_processor_count
-        alu_peak = sms * 128 * 2 * (clk["sm_max_mhz"] if clk and clk.get("sm_max_mhz") else 1965.0) * 1e6 / 1e12
+        # the chunkwise form on the tensor cores (dk = dv = 128): per chunk of
+        # C = 64 tokens, TF32 MMAs [Kt;Qt] Kh^T (128x64x128), S'^T [Kt;Qt]^T
+        # (128x128x128), U^T (128x64x64), O^T (128x64x64), S^T (128x128x64)
+        C = 64
+        mma = 2.0 * (128 * 64 * wl.dk + 128 * 128 * wl.dk + 128 * 64 * C + 128 * 64 * C + 128 * 128 * C)
+        flops = mma * nh * math.ceil(Tp / C)
+        tf32_peak = float(peaks.get("bf16_tflops", 1590.0)) * (1.1 / 2.25)
+        # the token-recurrent count for comparison: decay (1), S'^T k and S'^T q
+        # (2 x 2), update (2) flops per state entry and token
+        rec = 7.0 * wl.dk * wl.dv * nh * Tp
         line["prefill"] = {
             "prompt_tokens": Tp, "value": whole_job_rate(nh * Tp, world, pms), "unit": "head-tokens/s",
-            "ms_per_launch": pms, "bound": "alu", "achieved_tflops": flops / (pms / 1e3) / 1e12,
-            "peak_tflops": alu_peak, "frac": flops / (pms / 1e3) / 1e12 / alu_peak,
-            "peak_source": f"{sms} SMs x 128 FP32 lanes x 2 flops x max SM clock"}
+            "ms_per_launch": pms, "bound": "tensor", "achieved_tflops": flops / (pms / 1e3) / 1e12,
+            "peak_tflops": tf32_peak, "frac": flops / (pms / 1e3) / 1e12 / tf32_peak,
+            "peak_source": f"{peak_kind} bf16_tflops x 1.1/2.25 (nominal TF32 / BF16 dense ratio)",
+            "mma_flops_per_launch": flops, "recurrent_equivalent_tflops": rec / (pms / 1e3) / 1e12,
+            "form": "chunkwise, 64-token chunks, TF32 tcgen05 MMAs"}
         del stp, prompt
         torch.cuda.empty_cache()
 

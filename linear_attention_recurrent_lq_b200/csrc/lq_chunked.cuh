@@ -52,26 +52,29 @@ constexpr uint32_t kTmemCols = 512;
 constexpr uint32_t kColS = 0, kColW = 128, kColY = 192, kColA = 256, kColU = 320;
 
 // Shared memory (from a 1024-aligned base): tile region X [64 KB] | tile
-// region K [32 KB] | staging: q, k, v rows [kChunk][in bytes] each, KDA
-// decay rows [kChunk][128] f32 (staged with bf16 inputs; with f32 inputs they
-// would not fit and are read from global memory) | control.
+// region K [32 KB] | gate products G [kChunk][128] f32 | staging: q, k rows
+// [kChunk][in bytes], and with bf16 inputs also v rows and the KDA decay rows
+// [kChunk][128] f32 (with f32 inputs those would not fit and are read from
+// global memory) | control.
 struct ChunkSmem {
-    uint32_t stage_q, stage_k, stage_v, stage_dec, ctl, total;
-    int dec_staged;
+    uint32_t gbuf, stage_q, stage_k, stage_v, stage_dec, ctl, total;
+    int v_staged, dec_staged;
 };
 
 __host__ __device__ inline ChunkSmem chunk_smem(int bf16, int kda) {
     constexpr uint32_t D = 128;
     ChunkSmem S;
     const uint32_t qkv = D * (bf16 ? 2u : 4u);
+    S.v_staged = bf16;
     S.dec_staged = kda && bf16;
-    S.stage_q = 98304u;
+    S.gbuf = 98304u;
+    S.stage_q = S.gbuf + kChunk * D * 4u;
     S.stage_k = S.stage_q + kChunk * qkv;
     S.stage_v = S.stage_k + kChunk * qkv;
-    S.stage_dec = S.stage_v + kChunk * qkv;
+    S.stage_dec = S.stage_v + (S.v_staged ? kChunk * qkv : 0u);
     S.ctl = align_up(S.stage_dec + (S.dec_staged ? kChunk * D * 4u : 0u), 128u);
-    // control: barriers [2] | tmem slot | n | beta [64] | alpha [64] | gate scale [128] | M [16][16]
-    S.total = S.ctl + 64u + 4u * (2u * kChunk + 128u) + 1024u + 1024u;  // + alignment slack
+    // control: barriers [2] | tmem slot | n | beta [64] | alpha [64] | gate scale [128] | M [3][16][16]
+    S.total = S.ctl + 64u + 4u * (2u * kChunk + 128u) + 3072u + 1024u;  // + alignment slack
     return S;
 }
 
@@ -87,34 +90,69 @@ __device__ __forceinline__ void unit_lower_inverse(const float *Lb, float *Tb, f
         float x[16];
 #pragma unroll
         for (int r = 0; r < 16; ++r) {
+            float lr[16];
+#pragma unroll
+            for (int s = 0; s < 16; s += 4) {
+                const float4 w = *reinterpret_cast<const float4 *>(Lb + (o + r) * kChunk + o + s);
+                lr[s] = w.x; lr[s + 1] = w.y; lr[s + 2] = w.z; lr[s + 3] = w.w;
+            }
             float acc = r == c ? 1.f : 0.f;
 #pragma unroll
             for (int s = 0; s < r; ++s)
-                if (s >= c) acc = fmaf(-Lb[(o + r) * kChunk + o + s], x[s], acc);
+                if (s >= c) acc = fmaf(-lr[s], x[s], acc);
             x[r] = r < c ? 0.f : acc;
         }
 #pragma unroll
         for (int r = 0; r < 16; ++r) Tb[(o + r) * kChunk + o + c] = x[r];
     }
     __syncthreads();
-    // off-diagonal blocks, nearest the diagonal first:
-    // T_ij = -T_ii sum_{k=j}^{i-1} A_ik T_kj
-    const int r = tid >> 4, c = tid & 15;
+    // off-diagonal blocks, nearest the diagonal first, the blocks of one
+    // level at once: T_ij = -T_ii sum_{k=j}^{i-1} A_ik T_kj  (Mb: [3][16][16])
 #pragma unroll 1
-    for (int d = 1; d < 4; ++d)
+    for (int d = 1; d < 4; ++d) {
+        const int nb = 4 - d;
+        for (int e = tid; e < nb * 256; e += kGroup) {
+            const int bj = e >> 8, r = (e >> 4) & 15, c = e & 15, bi = bj + d;
+            float m0 = 0.f, m1 = 0.f;
 #pragma unroll 1
-        for (int bj = 0; bj + d < 4; ++bj) {
-            const int bi = bj + d;
-            float m = 0.f;
-            for (int k = 16 * bj; k < 16 * bi; ++k) m = fmaf(Lb[(16 * bi + r) * kChunk + k], Tb[k * kChunk + 16 * bj + c], m);
-            Mb[r * 16 + c] = m;
-            __syncthreads();
-            float t = 0.f;
+            for (int k0 = 16 * bj; k0 < 16 * bi; k0 += 16) {
+                float lr[16], tc[16];
 #pragma unroll
-            for (int s = 0; s < 16; ++s) t = fmaf(Tb[(16 * bi + r) * kChunk + 16 * bi + s], Mb[s * 16 + c], t);
-            Tb[(16 * bi + r) * kChunk + 16 * bj + c] = -t;
-            __syncthreads();
+                for (int y = 0; y < 16; y += 4) {
+                    const float4 w = *reinterpret_cast<const float4 *>(Lb + (16 * bi + r) * kChunk + k0 + y);
+                    lr[y] = w.x; lr[y + 1] = w.y; lr[y + 2] = w.z; lr[y + 3] = w.w;
+                }
+#pragma unroll
+                for (int y = 0; y < 16; ++y) tc[y] = Tb[(k0 + y) * kChunk + 16 * bj + c];
+#pragma unroll
+                for (int y = 0; y < 16; y += 2) {
+                    m0 = fmaf(lr[y], tc[y], m0);
+                    m1 = fmaf(lr[y + 1], tc[y + 1], m1);
+                }
+            }
+            Mb[e] = m0 + m1;
         }
+        __syncthreads();
+        for (int e = tid; e < nb * 256; e += kGroup) {
+            const int bj = e >> 8, r = (e >> 4) & 15, c = e & 15, bi = bj + d;
+            float tr[16], mc[16];
+#pragma unroll
+            for (int y = 0; y < 16; y += 4) {
+                const float4 w = *reinterpret_cast<const float4 *>(Tb + (16 * bi + r) * kChunk + 16 * bi + y);
+                tr[y] = w.x; tr[y + 1] = w.y; tr[y + 2] = w.z; tr[y + 3] = w.w;
+            }
+#pragma unroll
+            for (int y = 0; y < 16; ++y) mc[y] = Mb[(bj << 8) + y * 16 + c];
+            float t0 = 0.f, t1 = 0.f;
+#pragma unroll
+            for (int y = 0; y < 16; y += 2) {
+                t0 = fmaf(tr[y], mc[y], t0);
+                t1 = fmaf(tr[y + 1], mc[y + 1], t1);
+            }
+            Tb[(16 * bi + r) * kChunk + 16 * bj + c] = -(t0 + t1);
+        }
+        __syncthreads();
+    }
 }
 
 template <int BITS, bool SLOTS>
@@ -142,7 +180,7 @@ __global__ void __launch_bounds__(kGroup, 1) chunk_prefill_kernel(PrefillArgs A)
     float *s_beta = reinterpret_cast<float *>(smem + SM.ctl + 64);
     float *s_alpha = s_beta + kChunk;
     float *s_gs = s_alpha + kChunk;   // per key channel: the gate scale of the state
-    float *s_M = s_gs + 128;          // 16 x 16 scratch
+    float *s_M = s_gs + 128;          // [3][16][16] scratch
     const uint32_t rx = smem_u32(RX), rk = smem_u32(RK);
 
     pdl_wait();
@@ -198,31 +236,35 @@ __global__ void __launch_bounds__(kGroup, 1) chunk_prefill_kernel(PrefillArgs A)
 #pragma unroll 1
     for (int t0 = 0; t0 < len;) {
         const int nt = min(kChunk, len - t0);  // tokens staged (the chunk may end earlier)
-        // ---- stage q, k, v (and KDA decays) of tokens t0 .. t0 + nt; beta, alpha
-        if (warp == 0) {
-            if (lane == 0)
-                mbar_arrive_expect_tx(bar_stage, (uint32_t)nt * (3u * qkv + (SM.dec_staged ? (uint32_t)D * 4u : 0u)));
-            __syncwarp();
-            for (int x = lane; x < nt; x += 32) {
-                const size_t r = in_row(t0 + x);
-                bulk_g2s(smem + SM.stage_q + (size_t)x * qkv, static_cast<const uint8_t *>(A.q) + r * qkv, qkv, bar_stage);
-                bulk_g2s(smem + SM.stage_k + (size_t)x * qkv, static_cast<const uint8_t *>(A.k) + r * qkv, qkv, bar_stage);
-                bulk_g2s(smem + SM.stage_v + (size_t)x * qkv, static_cast<const uint8_t *>(A.v) + r * qkv, qkv, bar_stage);
-                if (SM.dec_staged)
-                    bulk_g2s(smem + SM.stage_dec + (size_t)x * D * 4, A.decay + r * D, (uint32_t)D * 4u, bar_stage);
+        float *G = reinterpret_cast<float *>(smem + SM.gbuf);  // [kChunk][D] gate products
+        // ---- stage q, k (and v, KDA decays) of tokens t0 .. t0 + nt with
+        // 16-byte loads by every thread; beta, alpha
+        {
+            const int cpr = (int)(qkv >> 4);  // 16-byte pieces per row
+            const int nbuf = SM.v_staged ? 3 : 2;
+#pragma unroll 4
+            for (int x = tid; x < nbuf * nt * cpr; x += kGroup) {
+                const int bsel = x / (nt * cpr), rem = x - bsel * nt * cpr, r = rem / cpr, c = rem - r * cpr;
+                const void *src = bsel == 0 ? A.q : (bsel == 1 ? A.k : A.v);
+                const uint32_t dst = bsel == 0 ? SM.stage_q : (bsel == 1 ? SM.stage_k : SM.stage_v);
+                const uint4 w = __ldg(reinterpret_cast<const uint4 *>(static_cast<const uint8_t *>(src) + in_row(t0 + r) * qkv) + c);
+                *reinterpret_cast<uint4 *>(smem + dst + (size_t)r * qkv + 16 * c) = w;
+            }
+            if (SM.dec_staged) {
+#pragma unroll 4
+                for (int x = tid; x < nt * (D / 4); x += kGroup) {
+                    const int r = x / (D / 4), c = x - r * (D / 4);
+                    const float4 w = __ldg(reinterpret_cast<const float4 *>(A.decay + in_row(t0 + r) * D) + c);
+                    *reinterpret_cast<float4 *>(smem + SM.stage_dec + (size_t)r * D * 4 + 16 * c) = w;
+                }
+            }
+            if (tid < kChunk) {
+                const bool in = tid < nt;
+                s_beta[tid] = in ? A.beta[in_row(t0 + tid)] : 0.f;
+                s_alpha[tid] = (in && !F.kda) ? A.decay[in_row(t0 + tid)] : 1.f;
             }
         }
-        if (tid < kChunk) {
-            const bool in = tid < nt;
-            s_beta[tid] = in ? A.beta[in_row(t0 + tid)] : 0.f;
-            s_alpha[tid] = (in && !F.kda) ? A.decay[in_row(t0 + tid)] : 1.f;
-        }
-        const bool landed = mbar_wait_bounded(bar_stage, stage_phase & 1u);
-        ++stage_phase;
-        if (!__syncthreads_and(landed)) {
-            failed = true;
-            break;
-        }
+        __syncthreads();
         const float *dec = reinterpret_cast<const float *>(smem + SM.stage_dec);
         auto a_of = [&](int x, int i) -> float {
             return F.kda ? (SM.dec_staged ? dec[x * D + i] : A.decay[in_row(t0 + x) * D + i]) : s_alpha[x];
@@ -231,43 +273,62 @@ __global__ void __launch_bounds__(kGroup, 1) chunk_prefill_kernel(PrefillArgs A)
             return load_in(smem + base + (size_t)x * qkv, i, F.bf16_in);
         };
 
-        // ---- pass 1: chunk length (the first token whose gate product falls
-        // below the range ends the chunk)
+        // ---- gate products G[x][i] (tokens t0+1 .. t0+x) and the chunk
+        // length: the first token whose product falls below the range ends it
         if (tid < D) {
             float g = 1.f;
             int viol = nt;
-            for (int x = 1; x < nt; ++x) {
-                g *= a_of(x, tid);
-                if (!(g >= kMinChunkGate)) {
-                    viol = x;
-                    break;
+            G[tid] = 1.f;
+#pragma unroll 1
+            for (int x0 = 1; x0 < nt; x0 += 8) {
+                float av[8];
+#pragma unroll
+                for (int y = 0; y < 8; ++y) av[y] = x0 + y < nt ? a_of(x0 + y, tid) : 1.f;
+#pragma unroll
+                for (int y = 0; y < 8; ++y) {
+                    g *= av[y];
+                    if (x0 + y < nt) {
+                        G[(x0 + y) * D + tid] = g;
+                        if (viol == nt && !(g >= kMinChunkGate)) viol = x0 + y;
+                    }
                 }
             }
             if (viol < kChunk) atomicMin(s_n, viol);
         }
         __syncthreads();
         const int n = min(*s_n, nt);
+        // the state's scale at the chunk end: the last product, times the next
+        // chunk's first gate (applied to S and to Kbar)
+        if (tid < D) s_gs[tid] = G[(n - 1) * D + tid] * (t0 + n < len ? gate(t0 + n, tid) : 1.f);
+        // the next chunk's rows into L2 while this one runs (a prefetch moves
+        // no data the kernel relies on); threads 128.. are free here
+        if (tid >= D && tid < D + kChunk && t0 + n + (tid - D) < len) {
+            const size_t r = in_row(t0 + n + (tid - D));
+            bulk_prefetch_l2(static_cast<const uint8_t *>(A.q) + r * qkv, qkv);
+            bulk_prefetch_l2(static_cast<const uint8_t *>(A.k) + r * qkv, qkv);
+            bulk_prefetch_l2(static_cast<const uint8_t *>(A.v) + r * qkv, qkv);
+            if (F.kda) bulk_prefetch_l2(A.decay + r * D, (uint32_t)D * 4u);
+        }
 
-        // ---- pass 2: X = [Kt; Qt] (128 x 128) and Kh (64 x 128), K-major tiles
-        {
-            const int i = tid & 127;
-            const bool kside = tid < 128;
-            float g = 1.f;
-#pragma unroll 1
-            for (int x = 0; x < kChunk; ++x) {
-                if (x > 0 && x < n) g *= a_of(x, i);
-                if (kside) {
-                    const float kv = x < n ? in_of(SM.stage_k, x, i) : 0.f;
-                    *reinterpret_cast<float *>(RX + sw128_off(x, i, 128)) = to_tf32(kv * g);
-                    *reinterpret_cast<float *>(RK + sw128_off(x, i, 64)) = to_tf32(kv * __frcp_rn(g));
-                } else {
-                    const float qv = x < n ? in_of(SM.stage_q, x, i) : 0.f;
-                    *reinterpret_cast<float *>(RX + sw128_off(64 + x, i, 128)) = to_tf32(qv * g);
-                }
+        // ---- X = [Kt; Qt] (128 x 128) and Kh (64 x 128), K-major tiles; a
+        // task is one row and four consecutive key channels
+#pragma unroll 4
+        for (int e = tid; e < 2 * kChunk * (D / 4); e += kGroup) {
+            const int qside = e >= kChunk * (D / 4), ee = e - (qside ? kChunk * (D / 4) : 0);
+            const int x = ee >> 5, i = 4 * (ee & 31);
+            float4 g4 = make_float4(1.f, 1.f, 1.f, 1.f), v4 = make_float4(0.f, 0.f, 0.f, 0.f);
+            if (x < n) {
+                g4 = *reinterpret_cast<const float4 *>(G + x * D + i);
+                const uint32_t base = qside ? SM.stage_q : SM.stage_k;
+                v4 = make_float4(in_of(base, x, i), in_of(base, x, i + 1), in_of(base, x, i + 2), in_of(base, x, i + 3));
             }
-            // the state's scale at the chunk end: the last product, times the
-            // next chunk's first gate (applied here, to S and to Kbar)
-            if (kside) s_gs[i] = g * (t0 + n < len ? gate(t0 + n, i) : 1.f);
+            const float4 t4 = make_float4(to_tf32(v4.x * g4.x), to_tf32(v4.y * g4.y), to_tf32(v4.z * g4.z),
+                                          to_tf32(v4.w * g4.w));
+            *reinterpret_cast<float4 *>(RX + sw128_off(qside ? 64 + x : x, i, 128)) = t4;
+            if (!qside)
+                *reinterpret_cast<float4 *>(RK + sw128_off(x, i, 64)) =
+                    make_float4(to_tf32(v4.x * __frcp_rn(g4.x)), to_tf32(v4.y * __frcp_rn(g4.y)),
+                                to_tf32(v4.z * __frcp_rn(g4.z)), to_tf32(v4.w * __frcp_rn(g4.w)));
         }
         fence_async_smem();
         tc_fence_before();
@@ -298,20 +359,24 @@ __global__ void __launch_bounds__(kGroup, 1) chunk_prefill_kernel(PrefillArgs A)
                 float v[16];
                 const int c0 = 32 * chalf + 16 * q;
                 tmem_ld16(tlane + kColA + (uint32_t)c0, v);
-                if (j < 64) {
-                    const int t = j;
+                const int t = j & 63;
+                const float bt = s_beta[t];
 #pragma unroll
-                    for (int x = 0; x < 16; ++x) {
-                        const int s = c0 + x;
-                        Lb[t * kChunk + s] = (s < t && t < n) ? s_beta[t] * v[x] : 0.f;
-                    }
-                } else {
-                    const int t = j - 64;
-#pragma unroll
-                    for (int x = 0; x < 16; ++x) {
-                        const int s = c0 + x;
-                        *reinterpret_cast<float *>(RX + 49152 + sw128_off(t, s, 64)) =
-                            to_tf32((s <= t && t < n) ? v[x] : 0.f);
+                for (int x = 0; x < 16; x += 4) {
+                    const int s0 = c0 + x;
+                    float4 o;
+                    if (j < 64) {
+                        o.x = (s0 < t && t < n) ? bt * v[x] : 0.f;
+                        o.y = (s0 + 1 < t && t < n) ? bt * v[x + 1] : 0.f;
+                        o.z = (s0 + 2 < t && t < n) ? bt * v[x + 2] : 0.f;
+                        o.w = (s0 + 3 < t && t < n) ? bt * v[x + 3] : 0.f;
+                        *reinterpret_cast<float4 *>(Lb + t * kChunk + s0) = o;
+                    } else {
+                        o.x = to_tf32((s0 <= t && t < n) ? v[x] : 0.f);
+                        o.y = to_tf32((s0 + 1 <= t && t < n) ? v[x + 1] : 0.f);
+                        o.z = to_tf32((s0 + 2 <= t && t < n) ? v[x + 2] : 0.f);
+                        o.w = to_tf32((s0 + 3 <= t && t < n) ? v[x + 3] : 0.f);
+                        *reinterpret_cast<float4 *>(RX + 49152 + sw128_off(t, s0, 64)) = o;
                     }
                 }
             }
@@ -319,22 +384,31 @@ __global__ void __launch_bounds__(kGroup, 1) chunk_prefill_kernel(PrefillArgs A)
         __syncthreads();
         unit_lower_inverse(Lb, Tb, s_M, tid);
         // Tinv as the B operand of U^T = RHS^T Tinv^T (rows t, K = s)
-        for (int x = tid; x < kChunk * kChunk; x += kGroup) {
-            const int t = x >> 6, s = x & 63;
-            *reinterpret_cast<float *>(RX + 32768 + sw128_off(t, s, 64)) = to_tf32(Tb[x]);
+        for (int e = tid; e < kChunk * kChunk / 4; e += kGroup) {
+            const int t = e >> 4, s0 = 4 * (e & 15);
+            const float4 w = *reinterpret_cast<const float4 *>(Tb + t * kChunk + s0);
+            *reinterpret_cast<float4 *>(RX + 32768 + sw128_off(t, s0, 64)) =
+                make_float4(to_tf32(w.x), to_tf32(w.y), to_tf32(w.z), to_tf32(w.w));
         }
         // RHS^T (rows j, K = s): beta_s (v_s[j] - W_s[j])
         {
+            auto v_at = [&](int s_) -> float {
+                return SM.v_staged ? in_of(SM.stage_v, s_, j) : load_in(A.v, in_row(t0 + s_) * D + j, F.bf16_in);
+            };
 #pragma unroll 1
             for (int q = 0; q < 2; ++q) {
                 float w[16];
                 const int c0 = 32 * chalf + 16 * q;
                 tmem_ld16(tlane + kColW + (uint32_t)c0, w);
 #pragma unroll
-                for (int x = 0; x < 16; ++x) {
-                    const int s = c0 + x;
-                    const float r = s < n ? s_beta[s] * (in_of(SM.stage_v, s, j) - w[x]) : 0.f;
-                    *reinterpret_cast<float *>(RX + sw128_off(j, s, 128)) = to_tf32(r);
+                for (int x = 0; x < 16; x += 4) {
+                    float r[4];
+#pragma unroll
+                    for (int y = 0; y < 4; ++y) {
+                        const int s_ = c0 + x + y;
+                        r[y] = to_tf32(s_ < n ? s_beta[s_] * (v_at(s_) - w[x + y]) : 0.f);
+                    }
+                    *reinterpret_cast<float4 *>(RX + sw128_off(j, c0 + x, 128)) = make_float4(r[0], r[1], r[2], r[3]);
                 }
             }
         }
@@ -374,20 +448,23 @@ __global__ void __launch_bounds__(kGroup, 1) chunk_prefill_kernel(PrefillArgs A)
                 const int c0 = 32 * chalf + 16 * q;
                 tmem_ld16(tlane + kColU + (uint32_t)c0, u);
 #pragma unroll
-                for (int x = 0; x < 16; ++x)
-                    *reinterpret_cast<float *>(RK + sw128_off(j, c0 + x, 128)) = to_tf32(u[x]);
+                for (int x = 0; x < 16; x += 4)
+                    *reinterpret_cast<float4 *>(RK + sw128_off(j, c0 + x, 128)) =
+                        make_float4(to_tf32(u[x]), to_tf32(u[x + 1]), to_tf32(u[x + 2]), to_tf32(u[x + 3]));
             }
-            // Kbar[s][i] = k_s,i * (G_last,i / G_s,i) * (next gate): thread i
-            // takes tokens [32 half, +32), its gate product recomputed
-            const int i = tid & 127, s0 = 32 * (tid >> 7);
-            float g = 1.f;
-            for (int x = 1; x <= s0 && x < n; ++x) g *= a_of(x, i);
-            const float gl = s_gs[i];
-#pragma unroll 1
-            for (int x = s0; x < s0 + 32; ++x) {
-                if (x > s0 && x < n) g *= a_of(x, i);
-                const float kb = x < n ? in_of(SM.stage_k, x, i) * (gl * __frcp_rn(g)) : 0.f;
-                *reinterpret_cast<float *>(RX + sw128_off(i, x, 128)) = to_tf32(kb);
+            // Kbar[s][i] = k_s,i (G_last,i / G_s,i) (next gate); a task is one
+            // key channel and four consecutive tokens
+#pragma unroll 4
+            for (int e = tid; e < D * (kChunk / 4); e += kGroup) {
+                const int i = e & 127, s0 = 4 * (e >> 7);
+                const float gl = s_gs[i];
+                float r[4];
+#pragma unroll
+                for (int y = 0; y < 4; ++y) {
+                    const int s_ = s0 + y;
+                    r[y] = to_tf32(s_ < n ? in_of(SM.stage_k, s_, i) * (gl * __frcp_rn(G[s_ * D + i])) : 0.f);
+                }
+                *reinterpret_cast<float4 *>(RX + sw128_off(i, s0, 128)) = make_float4(r[0], r[1], r[2], r[3]);
             }
         }
         fence_async_smem();
