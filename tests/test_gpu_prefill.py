@@ -193,3 +193,43 @@ def test_one_token_prompts_and_empty_prompts():
     assert not outz.any() and not outz.isnan().any()
     assert torch.equal(z.buf, ini.buf)
     assert z.check() == 0 and st.check() == 0
+
+
+@pytest.mark.parametrize("name", ["gdn_int8", "kda_int8_f16_f32in"])
+def test_prefill_extreme_gates_split_chunks(name):
+    """Gates of 0 and gate products far below the chunk range (1e-13 on every
+    channel, 1e-30 on one key channel), over a prompt of several chunks with
+    ragged lengths: the chunkwise prefill ends a chunk before each such token
+    and stays within 2e-3 of the FP64 oracle."""
+    wl, bits = CASES[name]
+    T = 150
+    lens = [150, 63, 130, 1, 97]
+    d = I.draw(wl, T)
+    dec = d["decay"]
+    if wl.decay_kind == "kda":
+        dec[20, :, :, 7] = 0.0          # one channel's gate is 0
+        dec[70] = 1e-13                 # every channel, every head
+        dec[90, :, :, 3] = 1e-30
+        dec[0, 1, :, 5] = 0.0           # a zero gate on a row's first token
+    else:
+        dec[20] = 0.0
+        dec[70] = 1e-13
+        dec[0, 1] = 0.0
+    st = _state(wl, bits)
+    nh, H = wl.batch * wl.heads, wl.heads
+    out = torch.empty((wl.batch, T, H, wl.dv), dtype=torch.float32, device="cuda")
+    S_fin = torch.empty((wl.batch, H, wl.dk, wl.dv), dtype=torch.float32, device="cuda")
+    lengths = torch.tensor(lens, dtype=torch.int32, device="cuda")
+    st.prefill(T, *_row_major(wl, d, T), S0=torch.from_numpy(d["S0"]).cuda(), lengths=lengths,
+               out=out, S_final=S_fin)
+    torch.cuda.synchronize()
+    p = _params(wl, bits)
+    o_ref, S_ref, _ = oracle.prefill(p, *oracle_inputs(wl, d, np.arange(nh), T), lengths=np.repeat(lens, H))
+    o_gpu = out.transpose(0, 1).cpu().numpy().reshape(T, nh, wl.dv)
+    S_gpu = S_fin.cpu().numpy().reshape(nh, wl.dk, wl.dv)
+    for h in range(nh):
+        n = lens[h // H]
+        assert np.isfinite(o_gpu[:, h]).all() and not o_gpu[n:, h].any()
+        assert rel_l2(o_gpu[:n, h], o_ref[:n, h]) < REL_L2, (h, rel_l2(o_gpu[:n, h], o_ref[:n, h]))
+        assert rel_l2(S_gpu[h], S_ref[h]) < REL_L2, (h, rel_l2(S_gpu[h], S_ref[h]))
+    assert st.check() == 0
