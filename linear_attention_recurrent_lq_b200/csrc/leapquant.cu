@@ -10,6 +10,7 @@
 #include "leapquant.h"
 #include "lq_common.cuh"
 #include "lq_decode.cuh"
+#include "lq_multi.cuh"
 #include "lq_dense.cuh"
 #include "lq_flush.cuh"
 #include "lq_fp32.cuh"
@@ -119,14 +120,28 @@ int persistent_grid(K kernel, int threads, uint32_t smem, int work) {
     return (int)(work < cap ? work : cap);
 }
 
+// Largest dynamic shared memory a block of this device may opt into.
+int smem_optin_limit() {
+    int dev = 0, v = 0;
+    if (cudaGetDevice(&dev) != cudaSuccess ||
+        cudaDeviceGetAttribute(&v, cudaDevAttrMaxSharedMemoryPerBlockOptin, dev) != cudaSuccess)
+        return -1;
+    return v;
+}
+
 template <int D, int BITS>
 lq_status launch_decode(const lq_config &c, const DecodeArgs &a, cudaStream_t s) {
     const bool multi = a.tokens > 1;
-    const uint32_t smem = decode_smem_bytes(D, a.L, a.F, multi ? a.tokens : 1);
-    auto k = a.map.slots ? (multi ? decode_kernel<D, BITS, true, true, false> : decode_kernel<D, BITS, true, false, false>)
-                         : (multi ? decode_kernel<D, BITS, false, true, false>
-                                  : ((a.flags & kEarlyState) ? decode_kernel<D, BITS, false, false, true>
-                                                             : decode_kernel<D, BITS, false, false, false>));
+    const uint32_t smem = multi ? multi_smem_bytes(D, a.L, a.F, a.tokens) : decode_smem_bytes(D, a.L, a.F, 1);
+    const bool t4 = a.tokens <= 4;
+    auto k = a.map.slots ? (multi ? (t4 ? decode_tokens_kernel<D, BITS, true, 4> : decode_tokens_kernel<D, BITS, true, 8>)
+                                  : decode_kernel<D, BITS, true, false>)
+                         : (multi ? (t4 ? decode_tokens_kernel<D, BITS, false, 4> : decode_tokens_kernel<D, BITS, false, 8>)
+                                  : ((a.flags & kEarlyState) ? decode_kernel<D, BITS, false, true>
+                                                             : decode_kernel<D, BITS, false, false>));
+    const int lim = smem_optin_limit();
+    if (lim < 0) return LQ_ERR_CUDA;
+    if (smem > (uint32_t)lim) return LQ_ERR_UNSUPPORTED;
     cudaError_t e = allow_smem(k, smem);
     if (e != cudaSuccess) return LQ_ERR_CUDA;
     const int threads = D + 64;

@@ -75,8 +75,9 @@ __host__ __device__ inline DecodeStage decode_stage(const Layout &L, int D, int 
                                                     int kda, int tokens = 1) {
     DecodeStage S;
     S.pairs_at = L.codes_off;  // the prefix [0, codes_off) is copied as is
-    // pairs buffered before the launch plus those its earlier tokens append: at most W - 1
-    S.in_off = align_up(S.pairs_at + (uint32_t)(window - 1) * L.pair_bytes, 128);
+    // pairs buffered before the launch plus those its tokens append: at most
+    // W - 1 for one token; a multi-token launch also stages its last key
+    S.in_off = align_up(S.pairs_at + (uint32_t)(tokens > 1 ? window : window - 1) * L.pair_bytes, 128);
     S.qkv_bytes = align_up((uint32_t)D * (bf16 ? 2u : 4u), 16);
     S.dec_off = S.in_off + 3u * S.qkv_bytes * (uint32_t)tokens;
     S.aux_off = align_up(S.dec_off + (kda ? (uint32_t)D * 4u * (uint32_t)tokens : 0u), 16);
@@ -167,7 +168,7 @@ constexpr int kInfoRun = 0, kInfoCount = 1, kInfoNrow = 2, kInfoNcol = 3, kInfoB
 
 template <int D>
 __host__ __device__ constexpr uint32_t decode_fixed_smem() {
-    // barriers (6 x 8 at 0, 2 more at 64) + control (128) | chunk sums float2 [D/16][D+1] | prep buffers [2]
+    // barriers (6 x 8 at 0) + control (128) | chunk sums float2 [D/16][D+1] | prep buffers [2]
     // | dots float2 [kDotSlots] | producer batch [4*32]
     return align_up(128u + 8u * (D / 16) * (D + 1) + 2u * PrepBuf<D>::bytes + 8u * kDotSlots + 4u * 32u * 4u,
                     128u);
@@ -323,16 +324,13 @@ __device__ __forceinline__ float warp_sum(float x) {
     return x;
 }
 
-// SLOTS: work items reach their blobs through A.map.  MULTI: each work item
-// takes A.tokens consecutive tokens (inputs and outputs [rows, T, H, .]),
-// reading its compact state once; token t sees the pairs of tokens < t
-// through the stage, where the epilogue also appends them.  EARLY (plain
-// rows only, kEarlyState): the first two blobs' state is staged before the
-// wait on the previous kernel.  Separate instances, so the plain path
-// carries none of this.
-template <int D, int BITS, bool SLOTS, bool MULTI, bool EARLY>
-__global__ void __launch_bounds__(D + 64, (SLOTS || MULTI) ? 3 : 0) decode_kernel(DecodeArgs A) {
-    static_assert(!(EARLY && (SLOTS || MULTI)), "early staging is for plain rows");
+// SLOTS: work items reach their blobs through A.map.  EARLY (plain rows
+// only, kEarlyState): the first two blobs' state is staged before the wait
+// on the previous kernel.  Separate instances, so the plain path carries
+// none of this.  (Several tokens per work item: decode_tokens_kernel.)
+template <int D, int BITS, bool SLOTS, bool EARLY>
+__global__ void __launch_bounds__(D + 64, SLOTS ? 3 : 0) decode_kernel(DecodeArgs A) {
+    static_assert(!(EARLY && SLOTS), "early staging is for plain rows");
     constexpr int NC = D;            // consumer threads
     constexpr int LPR = D / 16;      // threads per row, one 16-key chunk each
     constexpr int RPT = D / 16;      // rows per thread (16 row groups)
@@ -349,23 +347,15 @@ __global__ void __launch_bounds__(D + 64, (SLOTS || MULTI) ? 3 : 0) decode_kerne
     const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
     const Layout L = A.L;
     const Flags F = A.F;
-    const int T = MULTI ? A.tokens : 1;
-    const DecodeStage SG = decode_stage(L, D, F.window, F.bf16_in, F.kda, T);
+    const DecodeStage SG = decode_stage(L, D, F.window, F.bf16_in, F.kda);
     const int G = gridDim.x;
     const int n_mine = (A.num_heads - (int)blockIdx.x + G - 1) / G;
     auto blob_of = [](const SlotMap &m, int h) { return SLOTS ? m.blob(h) : h; };
-    // input / output row of token t of work item h: ((h / H) T + t) H + h % H
-    auto tok_row = [&](size_t h, int t) -> size_t {
-        if (!MULTI) return h;
-        const int H = A.map.heads;
-        return h + ((size_t)((int)h / H) * (size_t)(T - 1) + (size_t)t) * (size_t)H;
-    };
 
     extern __shared__ __align__(128) uint8_t smem[];
     uint64_t *full = reinterpret_cast<uint64_t *>(smem);  // [2] stage landed
     uint64_t *empty = full + 2;                           // [2] consumers done with the stage
     uint64_t *pfull = empty + 2;                          // [2] prep of the step done
-    uint64_t *pempty = reinterpret_cast<uint64_t *>(smem + 64);  // [2] consumers done with a prep buffer (MULTI)
     volatile uint32_t *s_abort = reinterpret_cast<volatile uint32_t *>(smem + 120);
     float2 *s_part = reinterpret_cast<float2 *>(smem + 128);            // chunk sums [LPR][PSTR]
     uint8_t *s_pb = reinterpret_cast<uint8_t *>(s_part + LPR * PSTR);    // PrepBuf [2]
@@ -381,7 +371,6 @@ __global__ void __launch_bounds__(D + 64, (SLOTS || MULTI) ? 3 : 0) decode_kerne
             mbar_init(&full[s], 1);
             mbar_init(&empty[s], NC / 32);  // one arrival per consumer warp
             mbar_init(&pfull[s], 32);       // every lane of the prep warp
-            if (MULTI) mbar_init(&pempty[s], NC / 32);
         }
         *s_abort = 0u;
         fence_mbar_init();
@@ -455,10 +444,8 @@ __global__ void __launch_bounds__(D + 64, (SLOTS || MULTI) ? 3 : 0) decode_kerne
                 const int b = blob_of(A.map, (int)h);
                 s_bidx[lane] = (int)b;
                 s_cnt[lane] = b >= 0 ? *reinterpret_cast<const uint32_t *>(A.state + b * L.blob + kHdrCount) : 0u;
-                if (!MULTI) {
-                    s_pbeta[lane] = A.beta[h];
-                    s_palpha[lane] = F.kda ? 1.f : A.decay[h];
-                }
+                s_pbeta[lane] = A.beta[h];
+                s_palpha[lane] = F.kda ? 1.f : A.decay[h];
             }
             __syncwarp();
             if (lane == 0) {
@@ -472,32 +459,15 @@ __global__ void __launch_bounds__(D + 64, (SLOTS || MULTI) ? 3 : 0) decode_kerne
                     const size_t h = blockIdx.x + (size_t)it * G;
                     uint8_t *st = stages + (size_t)s * SG.bytes;
                     float *aux = reinterpret_cast<float *>(st + SG.aux_off);
-                    if (!MULTI) {
-                        aux[4] = s_pbeta[x];
-                        aux[5] = s_palpha[x];
-                    } else {
-                        float bt[kMaxTokens], at[kMaxTokens];
-#pragma unroll
-                        for (int t = 0; t < kMaxTokens; ++t)
-                            if (t < T) {
-                                const size_t r = tok_row(h, t);
-                                bt[t] = A.beta[r];
-                                at[t] = F.kda ? 1.f : A.decay[r];
-                            }
-#pragma unroll
-                        for (int t = 0; t < kMaxTokens; ++t)
-                            if (t < T) {
-                                aux[4 + t] = bt[t];
-                                aux[4 + T + t] = at[t];
-                            }
-                    }
+                    aux[4] = s_pbeta[x];
+                    aux[5] = s_palpha[x];
                     aux[0] = s_bidx[x] >= 0 ? 0.f : 1.f;  // 1: no blob for this work item
                     if (s_bidx[x] < 0) {
                         mbar_arrive_expect_tx(&full[s], 0u);  // nothing is staged
                         continue;
                     }
                     const uint8_t *blob = A.state + (size_t)s_bidx[x] * L.blob;
-                    const uint32_t in_bytes = (uint32_t)T * (3 * SG.qkv_bytes + (F.kda ? (uint32_t)D * 4u : 0u));
+                    const uint32_t in_bytes = 3 * SG.qkv_bytes + (F.kda ? (uint32_t)D * 4u : 0u);
                     if (EARLY && it < kDecodeStages) {
                         mbar_arrive(&full[s]);  // state and inputs are on their way already
                         continue;
@@ -509,17 +479,12 @@ __global__ void __launch_bounds__(D + 64, (SLOTS || MULTI) ? 3 : 0) decode_kerne
                         bulk_g2s(st, blob, L.codes_off, &full[s]);
                         if (pb) bulk_g2s(st + SG.pairs_at, blob + L.pairs_off, pb, &full[s]);
                     }
-                    for (int t = 0; t < T; ++t) {
-                        const size_t r = tok_row(h, t);
-                        const size_t qo = r * (size_t)SG.qkv_bytes;
-                        uint8_t *in = st + SG.in_off + (size_t)t * 3 * SG.qkv_bytes;
-                        bulk_g2s(in, static_cast<const uint8_t *>(A.q) + qo, SG.qkv_bytes, &full[s]);
-                        bulk_g2s(in + SG.qkv_bytes, static_cast<const uint8_t *>(A.k) + qo, SG.qkv_bytes, &full[s]);
-                        bulk_g2s(in + 2 * SG.qkv_bytes, static_cast<const uint8_t *>(A.v) + qo, SG.qkv_bytes,
-                                 &full[s]);
-                        if (F.kda)
-                            bulk_g2s(st + SG.dec_off + (size_t)t * D * 4, A.decay + r * D, (uint32_t)D * 4u, &full[s]);
-                    }
+                    const size_t qo = h * (size_t)SG.qkv_bytes;
+                    uint8_t *in = st + SG.in_off;
+                    bulk_g2s(in, static_cast<const uint8_t *>(A.q) + qo, SG.qkv_bytes, &full[s]);
+                    bulk_g2s(in + SG.qkv_bytes, static_cast<const uint8_t *>(A.k) + qo, SG.qkv_bytes, &full[s]);
+                    bulk_g2s(in + 2 * SG.qkv_bytes, static_cast<const uint8_t *>(A.v) + qo, SG.qkv_bytes, &full[s]);
+                    if (F.kda) bulk_g2s(st + SG.dec_off, A.decay + h * D, (uint32_t)D * 4u, &full[s]);
                 }
             }
             __syncwarp();
@@ -533,23 +498,14 @@ __global__ void __launch_bounds__(D + 64, (SLOTS || MULTI) ? 3 : 0) decode_kerne
         // lists, the new decay product, y = g . k and g . q, the new key in
         // the window-start frame, x = sm . y quantized per 16-key chunk to
         // int16, and k . q.  Lane l takes keys KPL*l .. KPL*l + KPL - 1.
-        // One step per (head, token); the decay product runs on in registers
-        // over the tokens of a head.
-        float gprev[KPL];
-        bool dead = false;  // a token of this head failed its range check
-        for (int step = 0; step < n_mine * T; ++step) {
-            const int it = MULTI ? step / T : step, t = MULTI ? step - it * T : 0;
+        for (int it = 0; it < n_mine; ++it) {
             const int s = it % kDecodeStages;
             const uint8_t *st = stages + (size_t)s * SG.bytes;
-            uint8_t *pb = s_pb + (step & 1) * PB::bytes;
+            uint8_t *pb = s_pb + (it & 1) * PB::bytes;
             uint32_t *info = reinterpret_cast<uint32_t *>(pb + PB::info);
-            if (t == 0 && !mbar_wait_bounded(&full[s], (uint32_t)(it / kDecodeStages) & 1u)) {
+            if (!mbar_wait_bounded(&full[s], (uint32_t)(it / kDecodeStages) & 1u)) {
                 if (lane == 0) *s_abort = 1u;
                 break;  // the consumers time out on their own wait
-            }
-            if (MULTI && step >= 2 && !mbar_wait_bounded(&pempty[step & 1], (uint32_t)((step >> 1) - 1) & 1u)) {
-                if (lane == 0) *s_abort = 1u;
-                break;
             }
             const uint4 hdr = *reinterpret_cast<const uint4 *>(st);  // count, status, ncomp, magic
             const uint32_t ncomp = hdr.z;
@@ -565,35 +521,33 @@ __global__ void __launch_bounds__(D + 64, (SLOTS || MULTI) ? 3 : 0) decode_kerne
             uint32_t newbits = 0;
             if (hdr.w != kMagic || ncomp > (uint32_t)F.num_comp || hdr.x > (uint32_t)F.window || badm)
                 newbits = LQ_DEV_CORRUPT;
-            else if (hdr.y == 0 && hdr.x + (uint32_t)T > (uint32_t)F.window)
-                newbits = LQ_DEV_WINDOW_FULL;  // the window has no room for the T pairs
+            else if (hdr.y == 0 && hdr.x >= (uint32_t)F.window)
+                newbits = LQ_DEV_WINDOW_FULL;  // the window has no room for the pair
             // a work item without a blob: the stage holds stale bytes, skip it
             if (reinterpret_cast<const float *>(st + SG.aux_off)[0] != 0.f) newbits = kSkipItem;
-            if (t == 0) dead = false;
-            bool run = hdr.y == 0 && newbits == 0 && !dead;
+            bool run = hdr.y == 0 && newbits == 0;
             if (newbits == kSkipItem) newbits = 0;
             float kq = 0.f;
             if (run) {
                 const int i0 = KPL * lane;
-                const uint8_t *in = st + SG.in_off + (size_t)t * 3 * SG.qkv_bytes;
+                const uint8_t *in = st + SG.in_off;
                 float kv[KPL], qv[KPL], gn[KPL];
 #pragma unroll
                 for (int e = 0; e < KPL; ++e) {
                     kv[e] = load_in(in + SG.qkv_bytes, i0 + e, F.bf16_in);
                     qv[e] = load_in(in, i0 + e, F.bf16_in);
                 }
-                if (t == 0) {
+                float gprev[KPL];
 #pragma unroll
-                    for (int e = 0; e < KPL; ++e)
-                        gprev[e] = F.kda ? reinterpret_cast<const float *>(st + L.g_off)[i0 + e]
-                                         : *reinterpret_cast<const float *>(st + kHdrG);
-                }
+                for (int e = 0; e < KPL; ++e)
+                    gprev[e] = F.kda ? reinterpret_cast<const float *>(st + L.g_off)[i0 + e]
+                                     : *reinterpret_cast<const float *>(st + kHdrG);
                 if (F.kda) {
-                    const float *dec = reinterpret_cast<const float *>(st + SG.dec_off + (size_t)t * D * 4);
+                    const float *dec = reinterpret_cast<const float *>(st + SG.dec_off);
 #pragma unroll
                     for (int e = 0; e < KPL; ++e) gn[e] = gprev[e] * dec[i0 + e];
                 } else {
-                    const float alpha = reinterpret_cast<const float *>(st + SG.aux_off)[4 + T + t];
+                    const float alpha = reinterpret_cast<const float *>(st + SG.aux_off)[5];
 #pragma unroll
                     for (int e = 0; e < KPL; ++e) gn[e] = gprev[e] * alpha;
                 }
@@ -601,35 +555,23 @@ __global__ void __launch_bounds__(D + 64, (SLOTS || MULTI) ? 3 : 0) decode_kerne
                 // (rebase_frame): the stored parts take the factor and the
                 // product of those channels restarts at 1.  A negative or NaN
                 // gate is an input error (RANGE below).
-                bool small = false, invalid = false, rebase_timeout = false;
+                bool small = false, invalid = false;
 #pragma unroll
                 for (int e = 0; e < KPL; ++e) {
                     invalid |= !(gn[e] >= 0.f);
                     small |= gn[e] < kMinDecayProduct;
                 }
                 if (__any_sync(0xFFFFFFFFu, small) && !__any_sync(0xFFFFFFFFu, invalid)) {
-                    // inside one head, the consumers must be done with the previous
-                    // token (its pair is in the stage and the blob) first
-                    const bool waited = !(MULTI && t > 0) ||
-                                        mbar_wait_bounded(&pempty[(step - 1) & 1], (uint32_t)((step - 1) >> 1) & 1u);
-                    if (waited) {
-                        float f[KPL];
+                    float f[KPL];
 #pragma unroll
-                        for (int e = 0; e < KPL; ++e) f[e] = (!F.kda || gn[e] < kMinDecayProduct) ? gn[e] : 1.f;
-                        const int bh = blob_of(A.map, (int)(blockIdx.x + (size_t)it * G));
-                        rebase_frame<D>(const_cast<uint8_t *>(st), A.state + (size_t)bh * L.blob, L, SG.pairs_at,
-                                        hdr.x + (uint32_t)t, hdr.z, F.f16_scale, f, lane);
+                    for (int e = 0; e < KPL; ++e) f[e] = (!F.kda || gn[e] < kMinDecayProduct) ? gn[e] : 1.f;
+                    const int bh = blob_of(A.map, (int)(blockIdx.x + (size_t)it * G));
+                    rebase_frame<D>(const_cast<uint8_t *>(st), A.state + (size_t)bh * L.blob, L, SG.pairs_at, hdr.x,
+                                    hdr.z, F.f16_scale, f, lane);
 #pragma unroll
-                        for (int e = 0; e < KPL; ++e)
-                            if (!F.kda || gn[e] < kMinDecayProduct) gn[e] = 1.f;
-                    } else {
-                        if (lane == 0) *s_abort = 1u;
-                        rebase_timeout = true;  // the head is skipped below
-                        gn[0] = __int_as_float(0x7FC00000);
-                    }
+                    for (int e = 0; e < KPL; ++e)
+                        if (!F.kda || gn[e] < kMinDecayProduct) gn[e] = 1.f;
                 }
-#pragma unroll
-                for (int e = 0; e < KPL; ++e) gprev[e] = gn[e];
                 bool bad = false;
                 float yk[KPL], yq[KPL], kh[KPL], xk[KPL], xq[KPL];
                 float mk = 0.f, mq = 0.f;
@@ -697,20 +639,19 @@ __global__ void __launch_bounds__(D + 64, (SLOTS || MULTI) ? 3 : 0) decode_kerne
                 kq = warp_sum(kq);
                 if (bad) {
                     run = false;
-                    dead = true;  // the later tokens of this head are skipped too
-                    newbits = rebase_timeout ? LQ_DEV_TIMEOUT : LQ_DEV_RANGE;
+                    newbits = LQ_DEV_RANGE;
                 }
             }
             if (lane == 0) {
                 info[kInfoRun] = run ? 1u : 0u;
-                info[kInfoCount] = hdr.x + (uint32_t)t;
+                info[kInfoCount] = hdr.x;
                 info[kInfoNrow] = (uint32_t)__popc(rowm);
                 info[kInfoNcol] = (uint32_t)__popc(colm);
                 info[kInfoBits] = newbits;
                 info[kInfoKq] = __float_as_uint(kq);
             }
             __syncwarp();
-            mbar_arrive(&pfull[step & 1]);
+            mbar_arrive(&pfull[it & 1]);
         }
         return;
     }
@@ -730,26 +671,25 @@ __global__ void __launch_bounds__(D + 64, (SLOTS || MULTI) ? 3 : 0) decode_kerne
     // the prep of the head), so the chunk sums and dot products of the
     // previous head are free by then; the stage goes back to the copy warp
     // when every consumer warp has arrived on its "empty" barrier.
-    for (int step = 0; step < n_mine * T; ++step) {
-        const int it = MULTI ? step / T : step, t = MULTI ? step - it * T : 0;
+    for (int it = 0; it < n_mine; ++it) {
         const int s = it % kDecodeStages;
-        const uint32_t ph = (uint32_t)(step >> 1) & 1u;  // phase of this step's prep barrier
+        const uint32_t ph = (uint32_t)(it >> 1) & 1u;  // phase of this head's prep barrier
         const uint8_t *st = stages + (size_t)s * SG.bytes;
-        const uint8_t *pb = s_pb + (step & 1) * PB::bytes;
+        const uint8_t *pb = s_pb + (it & 1) * PB::bytes;
         const size_t h = blockIdx.x + (size_t)it * G;
-        const size_t orow = tok_row(h, t);  // input / output row of this token
+        const size_t orow = h;  // input / output row of this work item
         const int bi = blob_of(A.map, (int)h);
         uint8_t *blob = A.state + (bi >= 0 ? (size_t)bi : 0) * L.blob;
-        // codes of the next work item to load, during the last token of this
-        // one (through a slot map: if it has a blob)
-        bool has_next = it + 1 < n_mine && t == T - 1;
+        // codes of the next work item to load (through a slot map: if it has
+        // a blob)
+        bool has_next = it + 1 < n_mine;
         const uint8_t *next_codes = code_base + (h + G) * (size_t)L.blob;
         if constexpr (SLOTS) {
             const int bn = has_next ? A.map.blob((int)h + G) : -1;
             has_next = bn >= 0;
             next_codes = code_base + (size_t)(has_next ? bn : 0) * L.blob;
         }
-        if (!consumer_sync_and(mbar_wait_bounded(&pfull[step & 1], ph), NC)) {
+        if (!consumer_sync_and(mbar_wait_bounded(&pfull[it & 1], ph), NC)) {
             // the data never arrived: record it on this blob and stop this CTA
             if (tid == 0) {
                 if (bi >= 0) set_status(blob, LQ_DEV_TIMEOUT);
@@ -857,7 +797,7 @@ __global__ void __launch_bounds__(D + 64, (SLOTS || MULTI) ? 3 : 0) decode_kerne
                 const float uj = up[(size_t)m * 2 * D];
                 ab = __ffma2_rn(s_dot[m], make_float2(uj, uj), ab);
             }
-            const float u = aux[4 + t] * (load_in(st + SG.in_off + ((size_t)t * 3 + 2) * SG.qkv_bytes, j, F.bf16_in) - ab.x);
+            const float u = aux[4] * (load_in(st + SG.in_off + 2 * SG.qkv_bytes, j, F.bf16_in) - ab.x);
             const float kq = __uint_as_float(info[kInfoKq]);
             A.out[orow * D + j] = fmaf(kq, u, ab.y);
             const float *pkh = reinterpret_cast<const float *>(pb + PB::kh);
@@ -865,13 +805,6 @@ __global__ void __launch_bounds__(D + 64, (SLOTS || MULTI) ? 3 : 0) decode_kerne
             float *pair = reinterpret_cast<float *>(blob + L.pairs_off + (size_t)count * L.pair_bytes);
             pair[D + j] = u;
             pair[tid] = pkh[tid];
-            if (MULTI && t < T - 1) {
-                // the later tokens of this head read the pair from the stage
-                float *sp = reinterpret_cast<float *>(const_cast<uint8_t *>(st) + SG.pairs_at +
-                                                      (size_t)count * L.pair_bytes);
-                sp[D + j] = u;
-                sp[tid] = pkh[tid];
-            }
             if (F.kda) reinterpret_cast<float *>(blob + L.g_off)[tid] = pg[tid];
             if (tid == 0) {
                 *reinterpret_cast<uint32_t *>(blob + kHdrCount) = count + 1;
@@ -887,10 +820,7 @@ __global__ void __launch_bounds__(D + 64, (SLOTS || MULTI) ? 3 : 0) decode_kerne
             if (tid == 0 && newbits) set_status(blob, newbits);
         }
         __syncwarp();
-        if (lane == 0) {
-            if (MULTI) mbar_arrive(&pempty[step & 1]);  // this warp is done with the prep buffer
-            if (t == T - 1) mbar_arrive(&empty[s]);     // ... and, after the last token, with stage s
-        }
+        if (lane == 0) mbar_arrive(&empty[s]);  // this warp is done with stage s
     }
 }
 
