@@ -210,7 +210,7 @@ LQ_API lq_status lq_check_status(const lq_config *cfg, const void *state, lq_str
  *   LQ_STEP_EARLY_STATE  no kernel that may still be running when this step
  *      starts writes `state`.  The library launches with programmatic
  *      dependent launch, so the step can start while the kernel enqueued just
- *      before it drains; it then stages its first blobs' compact state and
+ *      before it drains; it then stages its first blob's compact state and
  *      codes at once, and reads q, k, v, beta and decay only after that
  *      kernel has completed.  The promise holds when (a) the kernel just
  *      before this call does not write `state`, and (b) that kernel is not a
