@@ -28,9 +28,11 @@ def _cuda():
                                                 ("kda_int8_b128h32", 8, True)])
 def test_early_state_steps_equal_plain_steps(kind, bits, per_step):
     from linear_attention_recurrent_lq_b200 import binding as B
-    # 63 heads: several per CTA of the LeapQuant decode; with 1200 heads the
-    # dense kernels (one CTA per SM) walk several heads per CTA as well
-    wl = I.WORKLOADS[kind].replace(batch=7 if bits in (8, 6, 4) and not per_step else 40,
+    # 900 heads: two or three per CTA of the LeapQuant decode (three CTAs per
+    # SM), so the heads after the early-staged first one take the ordinary
+    # path; with 1200 heads the dense kernels (one CTA per SM) walk several
+    # heads per CTA as well
+    wl = I.WORKLOADS[kind].replace(batch=100 if bits in (8, 6, 4) and not per_step else 40,
                                    heads=9 if bits in (8, 6, 4) and not per_step else 30, window=8)
     L, T = 3, 12  # three layer-states taking turns; a flush after token 8
     draws = [I.InputStream(wl, stream=l) for l in range(L)]
