@@ -215,3 +215,40 @@ def test_multi_token_at_the_largest_window_and_compensator_count():
     torch.cuda.synchronize()
     assert torch.equal(a.buf, b.buf)
     assert b.check() == 0
+
+
+@pytest.mark.parametrize("kind,bits", [("gdn_int8_b64h32", 8), ("kda_int8_b128h32", 4)])
+def test_multi_token_with_several_heads_per_cta_bitwise(kind, bits):
+    """900 heads: two or three per CTA of the multi-token kernel, so the
+    prep warp runs a head ahead, stages and prep buffers are reused and the
+    next head's codes load during the current one; T = 4 and 3 (four-token
+    instance) and T = 5 (eight-token instance), across a flush, bitwise equal
+    to single-token calls."""
+    wl = W[kind].replace(batch=100, heads=9)
+    Wn = 8
+    plan = [4, 3, 1, "flush", 5, 3]
+    n_tok = sum(p for p in plan if p != "flush")
+    d = I.draw(wl, n_tok)
+    dev = device_inputs(wl, d)
+    S0 = torch.from_numpy(d["S0"]).cuda()
+    a, b = _state(wl, bits, Wn), _state(wl, bits, Wn)
+    a.init(S0)
+    b.init(S0)
+    t0 = 0
+    for p in plan:
+        if p == "flush":
+            a.flush()
+            b.flush()
+            continue
+        ref = torch.empty((p, wl.batch, wl.heads, wl.dv), dtype=torch.float32, device="cuda")
+        _single(a, dev, t0, p, ref)
+        out = torch.full((wl.batch, p, wl.heads, wl.dv), float("nan"), device="cuda")
+        if p == 1:
+            b.step(*[dev[x][t0] for x in NAMES], out[:, 0])
+        else:
+            b.steps(p, *_stack(dev, t0, p), out)
+        torch.cuda.synchronize()
+        assert torch.equal(out, ref.transpose(0, 1)), (kind, t0, p)
+        assert torch.equal(a.buf, b.buf), (kind, t0, p)
+        t0 += p
+    assert b.check() == 0

@@ -212,3 +212,53 @@ def test_prefix_cache_round_trip_with_eviction():
     assert torch.equal(v[5 * H:6 * H], sv[2 * H:3 * H])
     assert torch.equal(v[4 * H:5 * H], sv[1 * H:2 * H])
     assert not v[:4 * H].any()
+
+
+def test_subset_at_scale_equals_a_plain_run_bitwise():
+    """100 of 150 slots with 9 heads: 900 work items, two or three per CTA of
+    the decode and multi-token kernels and three or four per CTA of the flush,
+    so the slot instances walk several blobs per CTA; single-token steps, a
+    four-token step and two flushes, bitwise against a plain run."""
+    wl = W["gdn_int8_b64h32"].replace(batch=130, heads=9)
+    bits, N, T = 8, 150, 10
+    d = I.draw(wl, T)
+    dev = device_inputs(wl, d)
+    rng = np.random.default_rng(7)
+    sel = sorted(rng.choice(wl.batch, 100, replace=False).tolist())
+    slots = rng.choice(N, 100, replace=False).tolist()
+    full = _state(wl, bits, num_slots=N)
+    alone = _state(wl, bits, num_slots=len(sel))
+    full.buf.copy_(torch.randint(0, 256, full.buf.shape, dtype=torch.uint8, device="cuda"))
+    S0 = torch.from_numpy(d["S0"]).cuda()[sel].contiguous()
+    alone.init(S0)
+    sl = _i32(slots)
+    H = wl.heads
+    for n, s in enumerate(slots):
+        full.blobs()[s * H:(s + 1) * H] = alone.blobs()[n * H:(n + 1) * H]
+    untouched = [s for s in range(N) if s not in slots]
+    before = _blob_rows(full, untouched).clone()
+    names = ("q", "k", "v", "beta", "decay")
+    t = 0
+    for p in (1, 1, 1, 1, "flush", 4, "flush", 1, 1):
+        if p == "flush":
+            alone.flush()
+            full.flush_slots(sl)
+            continue
+        if p == 1:
+            args = [_rows(dev[x][t], sel) for x in names]
+            out_a = torch.empty((len(sel), H, wl.dv), dtype=torch.float32, device="cuda")
+            out_f = torch.full_like(out_a, float("nan"))
+            alone.step(*args, out_a)
+            full.step_slots(sl, *args, out_f)
+        else:
+            args = [torch.stack([dev[x][t + i][sel] for i in range(p)], dim=1).contiguous() for x in names]
+            out_a = torch.empty((len(sel), p, H, wl.dv), dtype=torch.float32, device="cuda")
+            out_f = torch.full_like(out_a, float("nan"))
+            alone.steps(p, *args, out_a)
+            full.steps_slots(sl, p, *args, out_f)
+        torch.cuda.synchronize()
+        assert torch.equal(out_f, out_a), t
+        assert torch.equal(_blob_rows(full, slots), alone.blobs()), t
+        t += p
+    assert torch.equal(_blob_rows(full, untouched), before)
+    assert alone.check() == 0
