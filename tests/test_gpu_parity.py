@@ -233,6 +233,25 @@ def test_fp32_state_kernel_matches_oracle():
         assert rel_l2(S_gpu, S_ref) < 1e-5
 
 
+@pytest.mark.parametrize("kind", ["gdn_int8_b64h32", "kda_int8_b128h32"])
+def test_fp32_state_kernel_at_scale_sampled_heads(kind):
+    """1200 heads: eight per CTA of the FP32 kernel (one CTA per SM), so its
+    ring of stages is reused across heads; 32 seeded heads against the
+    oracle over 12 tokens."""
+    from linear_attention_recurrent_lq_b200 import binding as B
+    wl = W[kind].replace(batch=40, heads=30)
+    T = 12
+    d = I.draw(wl, T)
+    o_gpu, st = run_gpu(wl, d, T, cfg=B.config_for(wl, bits=32))
+    nh = wl.batch * wl.heads
+    heads = np.sort(np.random.default_rng(5).choice(nh, 32, replace=False))
+    p = oracle.Params(**{**_params(wl).__dict__, "bits": 32})
+    o_ref, S_ref, _ = oracle.run(p, *oracle_inputs(wl, d, heads, T))
+    assert rel_l2(o_gpu.reshape(T, nh, wl.dv)[:, heads], o_ref) < 1e-5
+    S_gpu = st.dequant().cpu().numpy().reshape(nh, wl.dk, wl.dv)[heads]
+    assert rel_l2(S_gpu, S_ref) < 1e-5
+
+
 @pytest.mark.parametrize("key", ["gdn_int8_b64h32", "kda_int8_b128h32", "gdn_6bit_b256h32",
                                  "gdn_4bit_b256h32"])
 def test_full_size_sampled_heads(key):
