@@ -241,7 +241,11 @@ LQ_API lq_status lq_decode_step_ex(const lq_config *cfg, void *state, const void
  * whole (LQ_DEV_WINDOW_FULL, zero outputs).  If token t fails its range
  * check, tokens t.. of that (slot, head) are skipped (zero outputs) and the
  * state keeps the pairs of tokens < t.  bits 8/6/4 only (others:
- * LQ_ERR_UNSUPPORTED).  T = 1 is lq_decode_step.  Every token is committed;
+ * LQ_ERR_UNSUPPORTED); LQ_ERR_UNSUPPORTED too when the launch's shared
+ * memory (two stages of W pair slots and T tokens' inputs, plus per-token
+ * scratch) exceeds what a block of the device may use, which no
+ * configuration within the limits of lq_validate_config reaches on a B200.
+ * T = 1 is lq_decode_step.  Every token is committed;
  * to keep only an accepted prefix (speculative decoding), snapshot the rows
  * first with lq_copy_slots, restore the rows that rejected tokens and decode
  * their accepted prefix again. */
