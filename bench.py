@@ -511,7 +511,7 @@ def cpu_baseline(wl, layer_np, seconds, oracle):
     nh = wl.batch * wl.heads
     W = wl.window
 
-    def run(nheads, nwin):
+    def run(nheads, nwin, threads=0):
         heads = np.arange(nheads)
         T = W * nwin
         tile = lambda x: np.tile(x, (nwin,) + (1,) * (x.ndim - 1))
@@ -523,7 +523,7 @@ def cpu_baseline(wl, layer_np, seconds, oracle):
         dshape = (W, nh, wl.dk) if wl.decay_kind == "kda" else (W, nh)
         decay = tile(layer_np["decay"].reshape(dshape)[:, heads])
         t0 = time.perf_counter()
-        _, _, used = oracle.run(p, S0, q, k, v, beta, decay, threads=0)
+        _, _, used = oracle.run(p, S0, q, k, v, beta, decay, threads=threads)
         return time.perf_counter() - t0, used, nheads * T
 
     dt, used, n = run(min(nh, 64), 1)
@@ -532,10 +532,28 @@ def cpu_baseline(wl, layer_np, seconds, oracle):
     nwin = max(1, int(round(rate * seconds / (nheads * W))))
     nwin = min(nwin, 64)
     dt, used, n = run(nheads, nwin)
+    # one thread on a sample of about a second, for the per-core figure
+    n1 = min(nh, max(1, int(rate / max(used, 1) / W)))
+    dt1, _, m1 = run(n1, 1, threads=1)
     return {"value": n / dt, "unit": "head-tokens/s", "cores": used, "kind": "oracle",
             "sample": f"{nheads} heads of one layer x {W * nwin} tokens (its first window of "
                       f"{W} tokens repeated {nwin}x), FP64 C oracle, OpenMP over heads, "
-                      f"{dt:.1f} s"}
+                      f"{dt:.1f} s",
+            "one_thread": {"value": m1 / dt1, "unit": "head-tokens/s",
+                           "sample": f"{n1} heads x {W} tokens, {dt1:.2f} s"},
+            "cpu_model": cpu_model()}
+
+
+def cpu_model():
+    """The host CPU's model name, as /proc/cpuinfo gives it."""
+    try:
+        with open("/proc/cpuinfo") as fh:
+            for line in fh:
+                if line.startswith("model name"):
+                    return line.split(":", 1)[1].strip()
+    except OSError:
+        pass
+    return None
 
 
 def measure_config(name, args, torch, B, I, hbm, dist, world):
