@@ -1,6 +1,6 @@
 """Host-side arithmetic of bench.py: the byte model behind the roofline
 numerator (config 1 figures worked out field by field), the whole-job rate,
-rank seeding, and the comment-blind source hash."""
+rank seeding, the comment-blind source hash, and the CPU oracle leg."""
 import os
 import sys
 
@@ -85,3 +85,17 @@ def test_head_token_bytes_and_restore_bytes(bench, wl):
     # a prefix-cache hit reads and writes the compact part: header 20, meta 16,
     # qs 512, sm 512, compensators 2048, codes 16384
     assert bench.restore_bytes(wl) == 2 * (20 + 16 + 512 + 512 + 2048 + 16384)
+
+
+def test_cpu_baseline_reports_all_cores_and_one_thread(bench):
+    """The oracle leg on a small workload: the contract's keys, a one-thread
+    figure beside the all-core one, and the host CPU's model name."""
+    import oracle
+    from linear_attention_recurrent_lq_b200 import inputs as I
+    wl = I.WORKLOADS["gdn_int8_b64h32"].replace(batch=2, heads=4)
+    d = I.draw(wl, wl.window)
+    r = bench.cpu_baseline(wl, d, 0.2, oracle)
+    assert r["kind"] == "oracle" and r["unit"] == "head-tokens/s" and r["value"] > 0
+    assert r["cores"] >= 1 and "heads" in r["sample"]
+    assert r["one_thread"]["value"] > 0 and r["one_thread"]["unit"] == "head-tokens/s"
+    assert r["cpu_model"] is None or isinstance(r["cpu_model"], str)
