@@ -249,3 +249,19 @@ def test_binding_checks_tensors_before_any_call(B, monkeypatch):
     # raw addresses are the caller's responsibility and pass through
     B.lq_window_flush(cfg, 256, stream=0)
     assert calls == ["lq_window_flush"]
+
+
+@pytest.mark.parametrize("lang,std", [("c", "-std=c99"), ("c++", "-std=c++11")])
+def test_header_compiles_without_cuda_headers(lang, std):
+    """include/leapquant.h stands alone: plain C99 and C++11, strict warnings,
+    no CUDA header on the include path (the stream is an opaque type)."""
+    import shutil
+    import subprocess
+    cc = shutil.which("gcc" if lang == "c" else "g++")
+    if cc is None:
+        pytest.skip("no host compiler")
+    src = '#include "leapquant.h"\nint main(void) { lq_config c; (void)c; return (int)LQ_OK; }\n'
+    r = subprocess.run([cc, std, "-Wall", "-Wextra", "-pedantic", "-Werror", "-fsyntax-only",
+                        "-I", os.path.dirname(HEADER), "-x", lang, "-"],
+                       input=src, capture_output=True, text=True)
+    assert r.returncode == 0, r.stderr
